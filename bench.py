@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the hot path: window scoring -> selection -> compaction -> decode.
+
+One step = one pass of the whole path over one batch of synthetic input: score,
+select (and allocate), layout, compact, then `steps` decode steps (append +
+decode attention). Prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b] [--impl kvc|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (weak
+scaling, no data-path collective); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+from workloads import get, make_inputs
+
+METRIC = "decode-attn tokens/s"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def esize(wl):
+    return 4 if wl.dtype == "fp32" else 2
+
+
+def work_per_step(wl, counts):
+    """Algorithmic bytes / flops of each phase of one step (no padding, no second scoring pass)."""
+    es = esize(wl)
+    S, G, d, L, w = wl.n_slots, wl.G, wl.d, wl.L, wl.w
+    out = {}
+    if w > 0:
+        N = L
+        out["score_bytes"] = S * L * d * es + S * G * w * d * es + S * N * 4
+        out["score_flops"] = 2.0 * S * G * w * L * d
+    kept = int(np.sum(counts))
+    out["compact_bytes"] = kept * 2 * d * es * 2 + kept * 4
+    dec = []
+    for t in range(wl.steps):
+        rows = kept + S * (t + 1)
+        dec.append(rows * 2 * d * es + S * G * d * es + S * G * d * 4)
+    out["decode_bytes"] = dec
+    return out
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            p = torch.cuda.get_device_properties(device_index)
+            self.bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        except Exception:
+            self.bus = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.bus:
+            cmd += ["-i", self.bus]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle timing (CPU baseline / reference arm)
+_ORACLE_INPUTS = {}
+
+
+def oracle_sample(wl, budget_s: float, seed_slots=0):
+    """Time the oracle on whole slots (scoring, selection, all decode steps) until `budget_s`
+    seconds pass or the workload is done; returns (seconds, slots done, threads)."""
+    from threadpoolctl import threadpool_limits
+    from oracle.pipeline import run_workload
+    if wl.name not in _ORACLE_INPUTS:
+        _ORACLE_INPUTS[wl.name] = make_inputs(wl, "cpu")
+    inp = _ORACLE_INPUTS[wl.name]
+    S = wl.n_slots
+    order = list(range(S))
+    rng = np.random.default_rng(seed_slots)
+    rng.shuffle(order)
+    with threadpool_limits(limits=1):
+        budgets = None
+        t0 = time.perf_counter()
+        done = 0
+        for s in order:
+            if wl.policy == "zigzag":
+                # timing sample only: the allocation needs every slot's LMBA count, so the
+                # sampled slots keep the average budget
+                budgets = np.full(wl.n_layers, wl.avg_budget, dtype=np.int64)
+            run_workload(inp, slots=[s], budgets=budgets)
+            done += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+    return dt, done, 1
+
+
+def reference_arm(args, wl, rank, world):
+    if rank != 0:
+        return 0
+    tokens = wl.batch * wl.steps
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        dt, done, cores = oracle_sample(wl, args.ref_step_seconds, seed_slots=i)
+        if i >= args.warmup:
+            per_step.append(dt * wl.n_slots / done)
+    ms = 1000.0 * statistics.mean(per_step)
+    value = tokens / (ms / 1000.0)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "context": wl.L, "decode_steps": wl.steps,
+                   "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"each step: whole slots of the workload (score, select, all decode steps) "
+                                   f"for ~{args.ref_step_seconds:.0f} s, scaled to all {wl.n_slots} slots"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ CUDA arm
+def cuda_arm(args, wl, rank, world, local_rank):
+    import torch.distributed as dist
+    import sparse_decode_attention_window_b200 as kvc
+    from sparse_decode_attention_window_b200.pipeline import KvcPipeline
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    kvc.library()
+    wl_r = wl.scaled(seed=wl.seed + 100003 * rank)
+    inp = make_inputs(wl_r, dev)
+    pipe = KvcPipeline(wl_r, inp)
+    stream = torch.cuda.current_stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    n_dec = wl.steps
+    out_all = torch.empty((n_dec,) + tuple(pipe.out.shape), dtype=torch.float32, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
+    e = [ev() for _ in range(4)]
+    ea = [ev() for _ in range(n_dec)]
+    ed = [ev() for _ in range(n_dec)]
+
+    def step_calls():
+        # one whole step of the hot path; the timing events become graph nodes
+        e[0].record()
+        pipe.score_step()
+        e[1].record()
+        pipe.select_step()
+        e[2].record()
+        pipe.compact_step()
+        e[3].record()
+        for t in range(n_dec):
+            kvc.kvc_append(pipe.shape, inp.k_dec[t], inp.v_dec[t], pipe.off, pipe.cap, pipe.len, pipe.kp, pipe.vp)
+            ea[t].record()
+            kvc.kvc_decode_attn(pipe.shape, inp.q_dec[t], pipe.kp, pipe.vp, pipe.off, pipe.len, out_all[t],
+                                pipe.ws_decode)
+            ed[t].record()
+
+    # eager warm-up: loads every kernel and sets its attributes before capture
+    for _ in range(max(1, args.warmup)):
+        flush.zero_()
+        step_calls()
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    counts = pipe.count.cpu().numpy()
+    work = work_per_step(wl, counts)
+
+    # the whole step as one CUDA graph (launch-bound decode loop: 2 launches per token step)
+    graph = torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream(device=dev)
+    cap_stream.wait_stream(torch.cuda.current_stream())
+    n0 = kvc.kvc_launch_count()
+    with torch.cuda.graph(graph, stream=cap_stream):
+        step_calls()
+    launches_per_step = kvc.kvc_launch_count() - n0
+    torch.cuda.current_stream().wait_stream(cap_stream)
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    step_ms, score_ms, select_ms, compact_ms, dec_ms, app_ms = [], [], [], [], [], []
+    for _ in range(args.steps):
+        flush.zero_()          # L2 flushed between steps, outside the timed events
+        graph.replay()
+        torch.cuda.synchronize()
+        score_ms.append(e[0].elapsed_time(e[1]))
+        select_ms.append(e[1].elapsed_time(e[2]))
+        compact_ms.append(e[2].elapsed_time(e[3]))
+        step_ms.append(e[0].elapsed_time(ed[-1]))
+        prev = e[3]
+        for t in range(n_dec):
+            app_ms.append(prev.elapsed_time(ea[t]))
+            dec_ms.append(ea[t].elapsed_time(ed[t]))
+            prev = ed[t]
+    torch.cuda.synchronize()
+    barrier()
+    launches = launches_per_step * args.steps
+    clk = clocks.stop()
+    kvc.kvc_get_status()
+
+    ms_step = statistics.mean(step_ms)
+    t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step_max = float(t.item())
+
+    # ---- end to end through the public API with host buffers
+    e2e = e2e_run(args, wl_r, inp, graph, out_all, dev)
+
+    # ---- CPU baseline (rank 0, single GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, done, cores = oracle_sample(wl, args.cpu_seconds)
+        full = dt * wl.n_slots / done
+        cpu = {"value": wl.batch * wl.steps / full, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{done} of {wl.n_slots} slots (score, select, {wl.steps} decode steps each) in "
+                         f"{dt:.1f} s on 1 thread, scaled to the whole step ({full:.1f} s)"}
+
+    del graph
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    dec_bytes = statistics.mean(work["decode_bytes"])
+    dec_us = 1000.0 * statistics.mean(dec_ms)
+    dec_gbs = dec_bytes / (dec_us * 1e-6) / 1e9
+    tokens_per_step = wl.batch * wl.steps
+    value = world * tokens_per_step / (ms_step_max / 1000.0)
+    ssc_us = 1000.0 * (statistics.mean(score_ms) + statistics.mean(select_ms) + statistics.mean(compact_ms))
+    phases = {
+        "score_us": 1000.0 * statistics.mean(score_ms),
+        "select_us": 1000.0 * statistics.mean(select_ms),
+        "compact_us": 1000.0 * statistics.mean(compact_ms),
+        "append_us_mean": 1000.0 * statistics.mean(app_ms),
+        "decode_us_mean": dec_us,
+    }
+    if "score_bytes" in work:
+        s_us = phases["score_us"]
+        phases["score_hbm_gbs"] = work["score_bytes"] / (s_us * 1e-6) / 1e9
+        phases["score_tflops"] = work["score_flops"] / (s_us * 1e-6) / 1e12
+        phases["score_tensor_frac_of_measured"] = phases["score_tflops"] / float(peaks["bf16_tflops"])
+    phases["compact_gbs"] = work["compact_bytes"] / (phases["compact_us"] * 1e-6) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.d,
+                   "context": wl.L, "window": wl.w, "policy": wl.policy, "decode_steps": wl.steps,
+                   "layers": wl.n_layers, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (2x L2 write) before every step, outside the timed events; "
+                         "within a step the compacted cache is re-read by each decode step"},
+        "decode_tokens_per_s": wl.batch / ((statistics.mean(app_ms) + statistics.mean(dec_ms)) / 1000.0) * world,
+        "decode_hbm_gbs": dec_gbs,
+        "score_select_compact_us_per_layer": ssc_us / wl.n_layers,
+        "phases": phases,
+        "roofline": {"kernel": "kvc_decode_attn", "bound": "hbm", "achieved": dec_gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": dec_gbs / hbm, "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": dec_bytes},
+        "clocks": clk,
+        "gpu_launches": int(launches),
+        "launches_per_step": int(launches_per_step),
+        "timing": "each step is one CUDA-graph replay of the C-ABI calls; phase and per-launch times from "
+                  "external CUDA events captured between the calls",
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def e2e_run(args, wl, inp, graph, out_all, dev):
+    """Same metric through the public API with host (pinned) buffers: each step copies its
+    inputs host -> device, runs the captured step (the C-ABI calls), and copies every
+    decode output back to the host."""
+    names = ["q_win", "k", "v", "q_dec", "k_dec", "v_dec", "special_mask", "chunk_end"]
+    host = {n: getattr(inp, n).cpu().pin_memory() for n in names if getattr(inp, n) is not None}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    out_host = torch.empty(tuple(out_all.shape), dtype=torch.float32).pin_memory()
+    d2h = out_host.numel() * 4
+    n = max(1, min(args.steps, args.e2e_steps))
+    times = []
+    for i in range(n + 1):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for nm, t in host.items():
+            getattr(inp, nm).copy_(t, non_blocking=True)
+        graph.replay()
+        out_host.copy_(out_all, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        if i > 0:            # first pass warms the copies
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.mean(times)
+    return {"value": wl.batch * wl.steps / (ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": n}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override a workload field (profiling cases), e.g. --set n_layers=8")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = get(args.workload)
+    for kv in args.set:
+        k, v = kv.split("=", 1)
+        cur = getattr(wl, k)
+        wl = wl.scaled(**{k: type(cur)(v)})
+    if args.impl == "reference":
+        return reference_arm(args, wl, rank, world)
+    return cuda_arm(args, wl, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

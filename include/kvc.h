@@ -1,0 +1,225 @@
+/*
+ * kvc.h - C ABI of the attention-score-driven KV eviction and ragged decode
+ * attention library (libkvc.so, sm_100a).
+ *
+ * The hot path, in call order:
+ *   kvc_score          window scoring (token keys or chunk keys)
+ *   kvc_select         per-head budget selection (top-B, LMBA mass count, FastGen
+ *                      local / special / full, ChunkLLM chunk selection)
+ *   kvc_alloc_budgets  ZigZagKV bounded per-layer budgets from the LMBA counts
+ *   kvc_layout         packed-cache offsets and capacities
+ *   kvc_compact        gather of the kept rows into the packed per-head cache
+ *   kvc_append         one new token per slot per decode step
+ *   kvc_decode_attn    split-K GQA decode attention over the ragged packed cache
+ *
+ * Sources: "ZigZagKV: Dynamic KV Cache Compression for Long-context Modeling based
+ * on Layer Uncertainty" (arXiv 2412.09036) Eq. 3-7; "Model Tells You What to
+ * Discard: Adaptive KV Cache Compression for LLMs" (FastGen, arXiv 2310.01801),
+ * abstract and Section 1; "ChunkLLM: A Lightweight Pluggable Framework for
+ * Accelerating LLMs Inference" (arXiv 2510.02361) Section 2.2, Eq. 3.
+ *
+ * Conventions (all calls):
+ *  - A slot is one (layer, batch row, KV head). Slots are numbered row-major in
+ *    that order; query head j of slot s is global query row s*G + j (GQA group G).
+ *  - Every tensor pointer is DEVICE memory owned by the caller; tensors are
+ *    contiguous, row-major, and 16-byte aligned. The library allocates no device
+ *    memory and keeps no state besides a per-device error word (read by
+ *    kvc_get_status) and a thread-local message (kvc_last_error).
+ *  - Calls are asynchronous on `stream`. Shapes and arguments are validated on the
+ *    host before any launch; a failed validation returns a non-zero kvc_status,
+ *    launches nothing, and sets the message. Device-side range checks never trap:
+ *    they skip the offending access and set a bit of the error word.
+ *  - Workspaces: `ws`/`ws_bytes` is caller-owned scratch of at least
+ *    kvc_workspace_size(...) bytes. It must be zero-filled before its first use;
+ *    every call leaves it zero-filled again, so one allocation serves many calls.
+ *    Calls that share a workspace must be ordered on one stream.
+ *  - Supported: head_dim d in {64, 128}; K/V/Q in bf16 or fp32
+ *    (the same type for all three); decode needs G in {1, 2, 4}, scoring G*w <= 256;
+ *    all accumulation in fp32.
+ */
+#ifndef KVC_H_
+#define KVC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVC_OK = 0,
+  KVC_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum */
+  KVC_ERR_SHAPE = 2,         /* inconsistent sizes */
+  KVC_ERR_UNSUPPORTED = 3,   /* valid but not implemented (e.g. d = 96) */
+  KVC_ERR_CAPACITY = 4,      /* an output buffer is too small */
+  KVC_ERR_CUDA = 5,          /* a CUDA runtime call failed */
+  KVC_ERR_WORKSPACE = 6,     /* workspace missing or too small */
+  KVC_ERR_DEVICE = 7         /* kvc_get_status: a kernel reported a range/timeout fault */
+} kvc_status;
+
+typedef enum { KVC_BF16 = 0, KVC_FP32 = 1 } kvc_dtype;
+
+typedef enum {
+  KVC_POL_TOPB = 0,        /* keep the B highest-scoring tokens (B = budget[s]) */
+  KVC_POL_MASS_COUNT = 1,  /* LMBA count only: smallest k whose top-k mass >= mass * total */
+  KVC_POL_LOCAL = 2,       /* FastGen local head: keep [L - W, L), W = budget[s] */
+  KVC_POL_SPECIAL = 3,     /* FastGen special-token head: keep positions set in special_mask */
+  KVC_POL_FULL = 4,        /* FastGen global head: keep [0, L) */
+  KVC_POL_CHUNK = 5        /* ChunkLLM: keep the top chunks until >= budget[s] tokens */
+} kvc_policy;
+
+/* Bit values of the device error word returned through kvc_get_status. */
+#define KVC_DEVERR_APPEND_OVERFLOW 0x1u  /* append found len == cap: token dropped */
+#define KVC_DEVERR_INDEX_RANGE     0x2u  /* compact/select met an out-of-range index or row */
+#define KVC_DEVERR_WAIT_TIMEOUT    0x4u  /* a pipeline wait hit its iteration limit */
+#define KVC_DEVERR_WORKSPACE       0x8u  /* a kernel's work list exceeded its workspace */
+
+typedef struct {
+  int32_t n_slots;   /* S = n_layers * batch * n_kv_heads */
+  int32_t G;         /* query heads per KV head */
+  int32_t d;         /* head dim */
+  int32_t L;         /* context length (keys per slot before compaction) */
+  int32_t w;         /* observation window (window queries per query head); 0 if unused */
+  int32_t n_kv_heads;/* KV heads per (layer, batch row): slot s has batch row (s / n_kv_heads) % batch */
+  int32_t batch;     /* batch rows per layer */
+  int32_t dtype;     /* kvc_dtype of Q, K, V */
+} kvc_shape;
+
+/* Workspace selectors for kvc_workspace_size. */
+#define KVC_WS_SCORE  0
+#define KVC_WS_SELECT 1
+#define KVC_WS_DECODE 2
+
+/*
+ * kvc_score - observation-window importance scores (ZigZagKV Eq. 7, after SnapKV).
+ *   For slot s, query head j < G and window row i < w (row position L - w + i),
+ *   p_{j,i,.} = softmax over the keys the row sees (key position <= L - w + i) of
+ *   q_{j,i} . k / sqrt(d); score[s][n] = sum_{j,i} p_{j,i,n}.
+ *   Token keys (chunk_end == NULL): key n is k[s][n], position n, n < L.
+ *   Chunk keys (ChunkLLM Eq. 3): key n < C is k[s][chunk_end[n]] (the chunk's last
+ *   token), position chunk_end[n]; chunk_end strictly increasing, last = L - 1.
+ *
+ *   q_win     [S*G, w, d]  window queries (dtype)
+ *   k         [S, L, d]    keys (dtype)
+ *   chunk_end [C] int32 or NULL; C its length (ignored when NULL)
+ *   row_lse   [S*G*w] fp32 or NULL: natural-log softmax normaliser of each window
+ *             row (log sum_n exp(q.k_n/sqrt(d)) over visible keys) if the caller has
+ *             it from prefill; NULL: computed here (one extra pass over K).
+ *   score     [S, N] fp32 out, N = L (tokens) or C (chunks)
+ * Errors: UNSUPPORTED for d not in {64,128} or G*w > 256; WORKSPACE if ws_bytes <
+ * kvc_workspace_size(KVC_WS_SCORE, shape, C).
+ */
+kvc_status kvc_score(const kvc_shape* shape, const void* q_win, const void* k,
+                     const int32_t* chunk_end, int32_t C, const float* row_lse,
+                     float* score, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * kvc_select - per-slot selection; each slot follows policy[s].
+ *   TOPB       keep budget[s] tokens with the highest score (ties: lower index first)
+ *   MASS_COUNT count[s] = LMBA of the slot (ZigZagKV Eq. 3): smallest k whose k
+ *              highest scores hold >= mass * (sum of scores); idx not written
+ *   LOCAL      keep [L - budget[s], L)
+ *   SPECIAL    keep n where special_mask[b][n] != 0, b the slot's batch row
+ *   FULL       keep [0, L)
+ *   CHUNK      `score` holds chunk scores [S, C]; keep the highest-scoring chunks
+ *              (ties: lower chunk index) until they hold >= budget[s] tokens,
+ *              emitting every token of the kept chunks
+ *   Kept indices are written to idx[s][0 .. count[s]) in ascending position order.
+ *
+ *   score        [S, N] fp32 (N = L, or C for CHUNK); may be NULL if no slot needs it
+ *   policy       [S] int8 kvc_policy, device
+ *   budget       [S] int32, device (B, W or token target; unused for MASS/SPECIAL/FULL)
+ *   special_mask [batch, L] uint8 or NULL (required if any slot is SPECIAL)
+ *   chunk_end    [C] int32 or NULL (required if any slot is CHUNK)
+ *   idx          [S, max_sel] int32 out; max_sel >= every count (else the kernel
+ *                clips, sets KVC_DEVERR_INDEX_RANGE)
+ *   count        [S] int32 out
+ */
+kvc_status kvc_select(const kvc_shape* shape, const float* score, const int8_t* policy,
+                      const int32_t* budget, float mass, const uint8_t* special_mask,
+                      const int32_t* chunk_end, int32_t C, int32_t* idx, int32_t max_sel,
+                      int32_t* count, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * kvc_alloc_budgets - ZigZagKV bounded per-layer budgets (Eq. 4-6).
+ *   C_l = sum of counts[l][0 .. spl); u_l = C_l / sum C; exact rational
+ *   B_l = floor_B + (avg_B - floor_B) * n_layers * u_l, made integer by floor plus
+ *   largest remainder (ties to the lower layer) so that sum B_l = n_layers * avg_B;
+ *   layers whose B_l exceeds L are fixed at L and the rest re-split the same way;
+ *   all-zero counts split uniformly.
+ *   counts       [n_layers * spl] int32 (MASS_COUNT of every slot), device
+ *   budgets      [n_layers] int32 out, device
+ *   slot_budgets [n_layers * spl] int32 out or NULL: B_l broadcast to each slot
+ * Errors: SHAPE unless 0 <= floor_B <= avg_B <= L.
+ */
+kvc_status kvc_alloc_budgets(const int32_t* counts, int32_t n_layers, int32_t spl, int32_t L,
+                             int32_t avg_B, int32_t floor_B, int32_t* budgets,
+                             int32_t* slot_budgets, cudaStream_t stream);
+
+/*
+ * kvc_layout - packed-cache layout: cap[s] = round_up(count[s] + reserve, 16);
+ *   off[0] = 0, off[s+1] = off[s] + cap[s] (rows). Slot s owns rows [off[s], off[s+1]).
+ *   count [S] int32 in; off [S+1] int64 out; cap [S] int32 out. All device.
+ */
+kvc_status kvc_layout(const int32_t* count, int32_t n_slots, int32_t reserve,
+                      int64_t* off, int32_t* cap, cudaStream_t stream);
+
+/*
+ * kvc_compact - kp[off[s] + r] = k[s][idx[s][r]], vp likewise, for r < count[s];
+ *   len[s] = count[s]. Rows [off[s] + count[s], off[s+1]) are not written.
+ *   k, v [S, L, d]; idx [S, max_sel]; kp, vp [kp_rows, d]; len [S] int32 out.
+ *   Rows outside [0, kp_rows) or indices outside [0, L) are skipped and flagged.
+ */
+kvc_status kvc_compact(const kvc_shape* shape, const void* k, const void* v,
+                       const int32_t* idx, int32_t max_sel, const int32_t* count,
+                       const int64_t* off, void* kp, void* vp, int64_t kp_rows,
+                       int32_t* len, cudaStream_t stream);
+
+/*
+ * kvc_append - one new token per slot: kp[off[s] + len[s]] = k_new[s], vp
+ *   likewise, len[s] += 1. A slot with len[s] == cap[s] (or whose next row would
+ *   fall outside the kp_rows rows of kp/vp) keeps its cache, leaves len unchanged
+ *   and sets KVC_DEVERR_APPEND_OVERFLOW.
+ *   k_new, v_new [S, d] (dtype); off [S+1]; cap, len [S]; kp, vp [kp_rows, d].
+ */
+kvc_status kvc_append(const kvc_shape* shape, const void* k_new, const void* v_new,
+                      const int64_t* off, const int32_t* cap, int32_t* len,
+                      void* kp, void* vp, int64_t kp_rows, cudaStream_t stream);
+
+/*
+ * kvc_decode_attn - for query head h of slot s = h / G:
+ *   out[h] = sum_{r < len[s]} softmax_r(q[h] . kp[off[s]+r] / sqrt(d)) vp[off[s]+r]
+ *   (fp32 accumulation and output). Work is split evenly over the GPU by token
+ *   ranges that may cross slot boundaries; partial results are merged by the last
+ *   CTA to finish a slot. A slot with len 0 yields zeros.
+ *   q [S*G, d] (dtype); kp, vp packed cache [kp_rows, d]; off [S+1]; len [S];
+ *   out [S*G, d] fp32. Rows past kp_rows are never read: a slot whose len runs past
+ *   them is cut short and KVC_DEVERR_INDEX_RANGE is set.
+ */
+kvc_status kvc_decode_attn(const kvc_shape* shape, const void* q, const void* kp,
+                           const void* vp, const int64_t* off, const int32_t* len,
+                           int64_t kp_rows, float* out, void* ws, size_t ws_bytes,
+                           cudaStream_t stream);
+
+/* Bytes of workspace the call `which` (KVC_WS_*) needs for this shape (C: chunks, 0 if none). */
+size_t kvc_workspace_size(int which, const kvc_shape* shape, int32_t C);
+
+/* Synchronises `stream`, reads and clears the current device's error word.
+ * Returns KVC_ERR_DEVICE (message names the bits) if it was non-zero. */
+kvc_status kvc_get_status(cudaStream_t stream);
+
+/* Message of the last failure on this host thread ("" if none). */
+const char* kvc_last_error(void);
+
+/* Library version string. */
+const char* kvc_version(void);
+
+/* Number of kernels this library has launched in this process so far (diagnostic). */
+unsigned long long kvc_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVC_H_ */

@@ -2,6 +2,7 @@
 
 The product path never imports this package.
 """
+from .oracle import _f64
 from .oracle import (window_scores, chunk_keys, chunk_scores, top_b, mass_count,
                      local_indices, special_indices, full_indices, chunk_select,
                      allocate_budgets, layout, compact, append, decode_attention)

@@ -1,0 +1,110 @@
+"""Attention-score-driven KV eviction and ragged decode attention for B200.
+
+Python face of libkvc.so (include/kvc.h): the functions below carry the C ABI's
+names and take torch CUDA tensors; they marshal pointers, sizes and the current
+stream and call the library, nothing more. The library must be built
+(`python -m sparse_decode_attention_window_b200.build`); without it every call
+raises - there is no CPU or PyTorch fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import (KvcShape, KvcError, KVC_BF16, KVC_FP32, KVC_POL_TOPB, KVC_POL_MASS_COUNT, KVC_POL_LOCAL,
+                   KVC_POL_SPECIAL, KVC_POL_FULL, KVC_POL_CHUNK, KVC_WS_SCORE, KVC_WS_SELECT, KVC_WS_DECODE)
+
+__all__ = ["KvcShape", "KvcError", "make_shape", "kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout",
+           "kvc_compact", "kvc_append", "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_version",
+           "kvc_launch_count",
+           "library", "KVC_BF16", "KVC_FP32", "KVC_POL_TOPB", "KVC_POL_MASS_COUNT", "KVC_POL_LOCAL",
+           "KVC_POL_SPECIAL", "KVC_POL_FULL", "KVC_POL_CHUNK", "KVC_WS_SCORE", "KVC_WS_SELECT", "KVC_WS_DECODE"]
+
+
+def library() -> ctypes.CDLL:
+    return _abi.load()
+
+
+def make_shape(n_slots, G, d, L, w=0, n_kv_heads=1, batch=1, dtype=torch.bfloat16) -> KvcShape:
+    dt = KVC_FP32 if dtype == torch.float32 else KVC_BF16
+    return KvcShape(int(n_slots), int(G), int(d), int(L), int(w), int(n_kv_heads), int(batch), dt)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("kvc: tensors must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("kvc: tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(name, rc):
+    if rc != 0:
+        raise KvcError(name, rc, library().kvc_last_error().decode())
+
+
+def kvc_workspace_size(which: int, shape: KvcShape, C: int = 0) -> int:
+    return int(library().kvc_workspace_size(which, ctypes.byref(shape), int(C)))
+
+
+def kvc_score(shape, q_win, k, score, ws, chunk_end=None, C=0, row_lse=None, stream=None):
+    _check("kvc_score", library().kvc_score(ctypes.byref(shape), _ptr(q_win), _ptr(k), _ptr(chunk_end), int(C),
+                                            _ptr(row_lse), _ptr(score), _ptr(ws), ws.numel() * ws.element_size(),
+                                            _stream(stream)))
+
+
+def kvc_select(shape, score, policy, budget, idx, count, mass=0.9, special_mask=None, chunk_end=None, C=0,
+               stream=None):
+    max_sel = idx.shape[-1] if idx is not None else 0
+    _check("kvc_select", library().kvc_select(ctypes.byref(shape), _ptr(score), _ptr(policy), _ptr(budget),
+                                              float(mass), _ptr(special_mask), _ptr(chunk_end), int(C), _ptr(idx),
+                                              int(max_sel), _ptr(count), None, 0, _stream(stream)))
+
+
+def kvc_alloc_budgets(counts, n_layers, spl, L, avg_B, floor_B, budgets, slot_budgets=None, stream=None):
+    _check("kvc_alloc_budgets", library().kvc_alloc_budgets(_ptr(counts), int(n_layers), int(spl), int(L),
+                                                            int(avg_B), int(floor_B), _ptr(budgets),
+                                                            _ptr(slot_budgets), _stream(stream)))
+
+
+def kvc_layout(count, reserve, off, cap, stream=None):
+    _check("kvc_layout", library().kvc_layout(_ptr(count), int(count.numel()), int(reserve), _ptr(off), _ptr(cap),
+                                              _stream(stream)))
+
+
+def kvc_compact(shape, k, v, idx, count, off, kp, vp, length, stream=None):
+    _check("kvc_compact", library().kvc_compact(ctypes.byref(shape), _ptr(k), _ptr(v), _ptr(idx), int(idx.shape[-1]),
+                                                _ptr(count), _ptr(off), _ptr(kp), _ptr(vp), int(kp.shape[0]),
+                                                _ptr(length), _stream(stream)))
+
+
+def kvc_append(shape, k_new, v_new, off, cap, length, kp, vp, stream=None):
+    _check("kvc_append", library().kvc_append(ctypes.byref(shape), _ptr(k_new), _ptr(v_new), _ptr(off), _ptr(cap),
+                                              _ptr(length), _ptr(kp), _ptr(vp), int(kp.shape[0]), _stream(stream)))
+
+
+def kvc_decode_attn(shape, q, kp, vp, off, length, out, ws, stream=None):
+    _check("kvc_decode_attn", library().kvc_decode_attn(ctypes.byref(shape), _ptr(q), _ptr(kp), _ptr(vp), _ptr(off),
+                                                        _ptr(length), int(kp.shape[0]), _ptr(out), _ptr(ws),
+                                                        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def kvc_get_status(stream=None):
+    _check("kvc_get_status", library().kvc_get_status(_stream(stream)))
+
+
+def kvc_version() -> str:
+    return library().kvc_version().decode()
+
+
+def kvc_launch_count() -> int:
+    return int(library().kvc_launch_count())

@@ -1,0 +1,201 @@
+// The packed per-head cache: layout (offsets by an exclusive scan of the
+// capacities), compaction (128-bit gathers of the kept K and V rows), the
+// per-step append, the gather of chunk keys, and the ZigZagKV per-layer budget
+// allocation (Eq. 4-6) that decides how many rows each layer keeps.
+#pragma once
+#include "common.cuh"
+
+namespace kvc {
+
+// ---------------------------------------------------------------- layout
+// One CTA: cap[s] = round_up(count[s] + reserve, 16); off = exclusive scan (int64).
+__global__ void __launch_bounds__(1024) layout_kernel(const int32_t* __restrict__ count, int S, int reserve,
+                                                      int64_t* __restrict__ off, int32_t* __restrict__ cap) {
+  __shared__ unsigned long long sh[33];
+  unsigned long long carry = 0;
+  for (int base = 0; base < S; base += blockDim.x) {
+    const int s = base + threadIdx.x;
+    unsigned long long c = 0;
+    if (s < S) {
+      long long want = (long long)max(count[s], 0) + reserve;
+      c = (unsigned long long)((want + 15) / 16 * 16);
+      cap[s] = (int32_t)c;
+    }
+    unsigned long long tot;
+    unsigned long long before = carry + block_exclusive_scan<unsigned long long>(c, sh, &tot);
+    if (s < S) off[s] = (int64_t)before;
+    carry += tot;
+  }
+  if (threadIdx.x == 0) off[S] = (int64_t)carry;
+}
+
+// ---------------------------------------------------------------- compaction
+// Persistent grid over the packed rows; a group of TPR = row_bytes/16 threads
+// copies one row of K and one of V with 16-byte loads and stores. The slot of a
+// packed row is found by binary search over off[].
+template <int TPR, int UNROLL>
+__global__ void __launch_bounds__(256) compact_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                                      const int32_t* __restrict__ idx, int max_sel,
+                                                      const int32_t* __restrict__ count,
+                                                      const int64_t* __restrict__ off, int S, int L,
+                                                      uint4* __restrict__ kp, uint4* __restrict__ vp,
+                                                      int64_t kp_rows, int32_t* __restrict__ len) {
+  const long long gthreads = (long long)gridDim.x * blockDim.x;
+  const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gtid < S) len[gtid] = min(max(count[gtid], 0), max_sel);
+  const int part = threadIdx.x % TPR;
+  const long long group = gtid / TPR, ngroups = gthreads / TPR;
+  const long long total = off[S];
+  for (long long g0 = group; g0 < total; g0 += ngroups * UNROLL) {
+    uint4 kr[UNROLL], vr[UNROLL];
+    long long dst[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      dst[u] = -1;
+      const long long g = g0 + (long long)u * ngroups;
+      if (g >= total) continue;
+      int lo = 0, hi = S - 1;            // last s with off[s] <= g
+      while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (off[mid] <= g) lo = mid; else hi = mid - 1;
+      }
+      const int s = lo;
+      const long long r = g - off[s];
+      const int cnt = min(count[s], max_sel);
+      if (r >= cnt) continue;            // padding row: not written
+      const int j = idx[(size_t)s * max_sel + r];
+      if (j < 0 || j >= L || g >= kp_rows) {
+        kvc_flag(KVC_DEVERR_INDEX_RANGE);
+        continue;
+      }
+      const size_t src = ((size_t)s * L + j) * TPR + part;
+      kr[u] = __ldg(k + src);
+      vr[u] = __ldg(v + src);
+      dst[u] = g * TPR + part;
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u)
+      if (dst[u] >= 0) {
+        kp[dst[u]] = kr[u];
+        vp[dst[u]] = vr[u];
+      }
+  }
+}
+
+// ---------------------------------------------------------------- append
+// grid S, block TPR: row off[s] + len[s] <- the new token; len[s] += 1.
+__global__ void append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                              const int64_t* __restrict__ off, const int32_t* __restrict__ cap,
+                              int32_t* __restrict__ len, uint4* __restrict__ kp, uint4* __restrict__ vp,
+                              int64_t kp_rows, int tpr) {
+  const int s = blockIdx.x;
+  const int n = len[s];
+  const bool ok = n >= 0 && n < cap[s] && off[s] + n < kp_rows;
+  if (ok) {
+    const size_t dst = ((size_t)off[s] + n) * tpr + threadIdx.x;
+    kp[dst] = k_new[(size_t)s * tpr + threadIdx.x];
+    vp[dst] = v_new[(size_t)s * tpr + threadIdx.x];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (ok) len[s] = n + 1;
+    else kvc_flag(KVC_DEVERR_APPEND_OVERFLOW);
+  }
+}
+
+// ---------------------------------------------------------------- chunk keys
+// kc[s][c] = k[s][chunk_end[c]] (ChunkLLM Eq. 3: a chunk is keyed by its last token).
+__global__ void gather_rows_kernel(const uint4* __restrict__ k, const int32_t* __restrict__ rows, int C, int L,
+                                   int S, int tpr, uint4* __restrict__ out) {
+  const long long total = (long long)S * C * tpr;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const long long row = e / tpr;
+    const int part = (int)(e - row * tpr);
+    const int s = (int)(row / C), c = (int)(row - (long long)s * C);
+    const int j = rows[c];
+    if (j < 0 || j >= L) { kvc_flag(KVC_DEVERR_INDEX_RANGE); continue; }
+    out[e] = k[((size_t)s * L + j) * tpr + part];
+  }
+}
+
+// ---------------------------------------------------------------- ZigZagKV allocation
+// One CTA of 1024 threads; n_layers <= 1024. Exact integer arithmetic.
+__global__ void __launch_bounds__(1024) alloc_kernel(const int32_t* __restrict__ counts, int nL, int spl, int L,
+                                                     int avg_B, int floor_B, int32_t* __restrict__ budgets,
+                                                     int32_t* __restrict__ slot_budgets) {
+  __shared__ long long Cl[1024];
+  __shared__ unsigned char capped[1024];
+  __shared__ long long rem[1024];
+  __shared__ long long base_[1024];
+  __shared__ unsigned long long red[33];
+  __shared__ int any_new;
+  const int tid = threadIdx.x;
+  for (int l = tid; l < nL; l += blockDim.x) {
+    long long c = 0;
+    for (int i = 0; i < spl; ++i) c += max(counts[(size_t)l * spl + i], 0);
+    Cl[l] = c;
+    capped[l] = 0;
+  }
+  __syncthreads();
+  const long long T = (long long)nL * avg_B;
+  const long long f = min(floor_B, L);
+  long long R = 0, E = 0, den = 0;
+  bool uniform = false;
+  int nU = 0;
+  while (true) {
+    // sums over the uncapped layers
+    unsigned long long my_c = 0, my_u = 0;
+    for (int l = tid; l < nL; l += blockDim.x)
+      if (!capped[l]) { my_c += (unsigned long long)Cl[l]; my_u += 1; }
+    const unsigned long long sumC = block_sum<unsigned long long>(my_c, red);
+    nU = (int)block_sum<unsigned long long>(my_u, red);
+    if (nU == 0) break;
+    R = T - (long long)(nL - nU) * L;
+    E = R - (long long)nU * f;
+    uniform = sumC == 0;
+    den = uniform ? nU : (long long)sumC;
+    if (tid == 0) any_new = 0;
+    __syncthreads();
+    for (int l = tid; l < nL; l += blockDim.x) {
+      if (capped[l]) continue;
+      const __int128 wl = uniform ? 1 : Cl[l];
+      // ideal = f + E * wl / den > L  <=>  f*den + E*wl > L*den
+      if ((__int128)f * den + (__int128)E * wl > (__int128)L * den) { capped[l] = 2; any_new = 1; }
+    }
+    __syncthreads();
+    const int again = any_new;
+    for (int l = tid; l < nL; l += blockDim.x)
+      if (capped[l] == 2) capped[l] = 1;
+    __syncthreads();
+    if (!again) break;
+  }
+  // floor + largest remainder over the uncapped layers (ties: lower layer)
+  unsigned long long my_b = 0;
+  for (int l = tid; l < nL; l += blockDim.x) {
+    if (capped[l]) continue;
+    const __int128 wl = uniform ? 1 : Cl[l];
+    const __int128 num = (__int128)f * den + (__int128)E * wl;
+    base_[l] = (long long)(num / den);
+    rem[l] = (long long)(num % den);
+    my_b += (unsigned long long)base_[l];
+  }
+  const long long sum_base = nU > 0 ? (long long)block_sum<unsigned long long>(my_b, red) : 0;
+  const long long left = R - sum_base;
+  for (int l = tid; l < nL; l += blockDim.x) {
+    long long b;
+    if (capped[l]) {
+      b = L;
+    } else {
+      long long rank = 0;
+      for (int m = 0; m < nL; ++m)
+        if (!capped[m] && (rem[m] > rem[l] || (rem[m] == rem[l] && m < l))) ++rank;
+      b = base_[l] + (rank < left ? 1 : 0);
+    }
+    budgets[l] = (int32_t)b;
+    if (slot_budgets)
+      for (int i = 0; i < spl; ++i) slot_budgets[(size_t)l * spl + i] = (int32_t)b;
+  }
+}
+
+}  // namespace kvc

@@ -1,0 +1,435 @@
+// libkvc: host side of the C ABI declared in include/kvc.h. Every entry point
+// validates its arguments on the host, picks a kernel and launches it on the
+// caller's stream; nothing here allocates device memory. All kernels live in
+// the headers included below (one translation unit, one device error word).
+#include <cstdio>
+#include <cstdarg>
+#include <cstdlib>
+#include <cstring>
+#include <atomic>
+#include <map>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "score_simt.cuh"
+#include "cache.cuh"
+#include "score_sm100.cuh"
+#include "select.cuh"
+#include "decode.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_launches{0};
+
+void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+kvc_status fail(kvc_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+kvc_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  g_last_error.clear();
+  return KVC_OK;
+}
+
+struct DevInfo {
+  int sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  int smem_optin = 0;
+};
+
+constexpr int kMaxDevices = 64;
+DevInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+
+kvc_status dev_info(DevInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(KVC_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::call_once(g_dev_once[dev], [dev] {
+    cudaDeviceGetAttribute(&g_dev[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&g_dev[dev].cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&g_dev[dev].cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&g_dev[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  });
+  *out = &g_dev[dev];
+  return KVC_OK;
+}
+
+// Opt a kernel in to `bytes` of dynamic shared memory. The attribute is set once per
+// (kernel, device) and raised only when a larger size is asked for, so repeated calls
+// (and calls made while a stream is being captured into a graph) do no driver work.
+std::mutex g_smem_mu;
+std::map<std::pair<const void*, int>, size_t> g_smem_set;
+
+template <typename K>
+kvc_status set_smem(K kernel, size_t bytes, const char* what) {
+  if (bytes <= 48 * 1024) return KVC_OK;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  auto it = g_smem_set.find(key);
+  if (it != g_smem_set.end() && it->second >= bytes) return KVC_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "%s: shared memory %zu B: %s", what, bytes, cudaGetErrorString(e));
+  g_smem_set[key] = bytes;
+  return KVC_OK;
+}
+
+size_t esize(int dtype) { return dtype == KVC_FP32 ? 4 : 2; }
+
+kvc_status check_shape(const kvc_shape* sh, bool need_window) {
+  if (!sh) return fail(KVC_ERR_INVALID_ARG, "shape is NULL");
+  if (sh->n_slots <= 0 || sh->G <= 0 || sh->d <= 0 || sh->L <= 0)
+    return fail(KVC_ERR_SHAPE, "n_slots, G, d, L must be positive (got %d, %d, %d, %d)", sh->n_slots, sh->G,
+                sh->d, sh->L);
+  if (sh->dtype != KVC_BF16 && sh->dtype != KVC_FP32) return fail(KVC_ERR_INVALID_ARG, "bad dtype %d", sh->dtype);
+  if (sh->d != 64 && sh->d != 128) return fail(KVC_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", sh->d);
+  if (need_window && (sh->w <= 0 || sh->w > sh->L))
+    return fail(KVC_ERR_SHAPE, "window w = %d must be in [1, L = %d]", sh->w, sh->L);
+  if (sh->n_kv_heads <= 0 || sh->batch <= 0) return fail(KVC_ERR_SHAPE, "n_kv_heads and batch must be positive");
+  return KVC_OK;
+}
+
+// KVC_SCORE_PATH=simt routes bf16 scoring to the CUDA-core kernels (used to cross-check
+// the two paths against each other); read once per process.
+bool force_simt() {
+  static const bool v = [] {
+    const char* e = getenv("KVC_SCORE_PATH");
+    return e && strcmp(e, "simt") == 0;
+  }();
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- workspace layouts
+struct ScoreWs {
+  size_t part_off, part_bytes;   // float2 partial row statistics
+  size_t lse_off, lse_bytes;     // float per window row
+  size_t keys_off, keys_bytes;   // gathered chunk keys (tensor-core path)
+  size_t total;
+};
+
+ScoreWs score_ws_layout(const kvc_shape* sh, int C, int sms) {
+  const int R = sh->G * sh->w;
+  const long long N = C > 0 ? C : sh->L;
+  const long long nblk_simt = (N + kvc::SIMT_TB - 1) / kvc::SIMT_TB;
+  const long long nsplit_tc = kvc::tc_num_splits(sh->n_slots, N, sms);
+  const long long nparts = nblk_simt > nsplit_tc ? nblk_simt : nsplit_tc;
+  ScoreWs w{};
+  w.part_off = 0;
+  w.part_bytes = align_up((size_t)sh->n_slots * nparts * R * sizeof(float2), 256);
+  w.lse_off = w.part_off + w.part_bytes;
+  w.lse_bytes = align_up((size_t)sh->n_slots * R * sizeof(float), 256);
+  w.keys_off = w.lse_off + w.lse_bytes;
+  w.keys_bytes = C > 0 ? align_up((size_t)sh->n_slots * C * sh->d * esize(sh->dtype), 256) : 0;
+  w.total = w.keys_off + w.keys_bytes;
+  return w;
+}
+
+struct DecodeWs {
+  size_t part_off, part_bytes, cnt_off, cnt_bytes, total;
+};
+
+DecodeWs decode_ws_layout(const kvc_shape* sh, int sms) {
+  DecodeWs w{};
+  w.cnt_off = 0;
+  w.cnt_bytes = align_up((size_t)sh->n_slots * sizeof(int), 256);
+  w.part_off = w.cnt_bytes;
+  w.part_bytes = align_up((size_t)(sms + sh->n_slots) * sh->G * (sh->d + 2) * sizeof(float), 256);
+  w.total = w.part_off + w.part_bytes;
+  return w;
+}
+
+// ---- decode dispatch
+template <typename T, int D, int G>
+kvc_status launch_decode(const kvc::DecodeParams& p, int sms, cudaStream_t st) {
+  using namespace kvc;
+  const size_t smem = decode_smem_bytes<T, D, G>(p.S);
+  DevInfo* di = nullptr;
+  if (dev_info(&di) != KVC_OK) return KVC_ERR_CUDA;
+  if (smem > (size_t)di->smem_optin)
+    return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: %d slots need %zu B of shared memory (> %d)", p.S, smem,
+                di->smem_optin);
+  kvc_status rc = set_smem(decode_kernel<T, D, G>, smem, "kvc_decode_attn");
+  if (rc != KVC_OK) return rc;
+  decode_kernel<T, D, G><<<sms, DecCfg<T, D, G>::THREADS, smem, st>>>(p);
+  count_launches(1);
+  return check_launch("kvc_decode_attn");
+}
+
+template <typename T, int D>
+kvc_status decode_by_g(int G, const kvc::DecodeParams& p, int sms, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode<T, D, 1>(p, sms, st);
+    case 2: return launch_decode<T, D, 2>(p, sms, st);
+    case 4: return launch_decode<T, D, 4>(p, sms, st);
+    default: return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: G = %d (supported: 1, 2, 4)", G);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvc_last_error(void) { return g_last_error.c_str(); }
+
+const char* kvc_version(void) { return "kvc 0.1 (sm_100a)"; }
+
+unsigned long long kvc_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t kvc_workspace_size(int which, const kvc_shape* shape, int32_t C) {
+  if (!shape || shape->n_slots <= 0) return 0;
+  DevInfo* di = nullptr;
+  int sms = 148;
+  if (dev_info(&di) == KVC_OK && di->sms > 0) sms = di->sms;
+  switch (which) {
+    case KVC_WS_SCORE: return score_ws_layout(shape, C, sms).total;
+    case KVC_WS_SELECT: return 0;
+    case KVC_WS_DECODE: return decode_ws_layout(shape, sms).total;
+    default: return 0;
+  }
+}
+
+kvc_status kvc_get_status(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  unsigned int word = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&word, g_kvc_deverr, sizeof(word));
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "read error word: %s", cudaGetErrorString(e));
+  if (word == 0) {
+    g_last_error.clear();
+    return KVC_OK;
+  }
+  cudaMemcpyToSymbol(g_kvc_deverr, &zero, sizeof(zero));
+  return fail(KVC_ERR_DEVICE, "device error word 0x%x:%s%s%s%s", word,
+              (word & KVC_DEVERR_APPEND_OVERFLOW) ? " append-overflow" : "",
+              (word & KVC_DEVERR_INDEX_RANGE) ? " index-out-of-range" : "",
+              (word & KVC_DEVERR_WAIT_TIMEOUT) ? " wait-timeout" : "",
+              (word & KVC_DEVERR_WORKSPACE) ? " workspace" : "");
+}
+
+kvc_status kvc_score(const kvc_shape* shape, const void* q_win, const void* k, const int32_t* chunk_end, int32_t C,
+                     const float* row_lse, float* score, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, true);
+  if (rc != KVC_OK) return rc;
+  if (!q_win || !k || !score) return fail(KVC_ERR_INVALID_ARG, "kvc_score: q_win, k and score must be non-NULL");
+  if (chunk_end && (C <= 0 || C > shape->L))
+    return fail(KVC_ERR_SHAPE, "kvc_score: chunk count C = %d must be in [1, L]", C);
+  const int R = shape->G * shape->w;
+  if (R > 256) return fail(KVC_ERR_UNSUPPORTED, "kvc_score: G*w = %d > 256", R);
+  DevInfo* di = nullptr;
+  if ((rc = dev_info(&di)) != KVC_OK) return rc;
+  const int Cc = chunk_end ? C : 0;
+  const ScoreWs w = score_ws_layout(shape, Cc, di->sms);
+  if (!ws || ws_bytes < w.total)
+    return fail(KVC_ERR_WORKSPACE, "kvc_score: workspace %zu B < required %zu B", ws_bytes, w.total);
+  if (!aligned16(q_win) || !aligned16(k) || !aligned16(ws))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_score: q_win, k and ws must be 16-byte aligned");
+  unsigned char* wsb = static_cast<unsigned char*>(ws);
+  float2* part = reinterpret_cast<float2*>(wsb + w.part_off);
+  float* lse = reinterpret_cast<float*>(wsb + w.lse_off);
+  const int N = chunk_end ? C : shape->L;
+  const float scale = 1.0f / sqrtf((float)shape->d);
+  const int S = shape->n_slots, d = shape->d;
+
+  if (kvc::tc_supported(shape, di->cc_major, di->cc_minor) && !force_simt()) {
+    unsigned nl = 0;
+    rc = kvc::tc_score(shape, q_win, k, chunk_end, C, row_lse, score, part, lse, wsb + w.keys_off, di->sms, stream,
+                       &fail, &nl);
+    count_launches(nl);
+    if (rc != KVC_OK) return rc;
+    return check_launch("kvc_score");
+  }
+
+  // CUDA-core path: stats + merge + column sums (or column sums alone given row_lse)
+  count_launches(row_lse ? 1 : 3);
+  const int nblk = (N + kvc::SIMT_TB - 1) / kvc::SIMT_TB;
+  const size_t sm1 = ((size_t)R * d + (size_t)kvc::SIMT_TB * (d + 1)) * sizeof(float);
+  const size_t sm2 = sm1 + (size_t)R * sizeof(float) + kvc::SIMT_THREADS * sizeof(float);
+  dim3 grid(nblk, S);
+  if (shape->dtype == KVC_FP32) {
+    const float* q = static_cast<const float*>(q_win);
+    const float* kk = static_cast<const float*>(k);
+    if (!row_lse) {
+      if ((rc = set_smem(kvc::score_stats_simt<float>, sm1, "kvc_score")) != KVC_OK) return rc;
+      kvc::score_stats_simt<float><<<grid, kvc::SIMT_THREADS, sm1, stream>>>(q, kk, chunk_end, N, shape->L,
+                                                                              shape->G, shape->w, d, scale, part);
+      kvc::score_lse_merge<<<S, 256, 0, stream>>>(part, nblk, R, lse);
+    }
+    if ((rc = set_smem(kvc::score_colsum_simt<float>, sm2, "kvc_score")) != KVC_OK) return rc;
+    kvc::score_colsum_simt<float><<<grid, kvc::SIMT_THREADS, sm2, stream>>>(
+        q, kk, chunk_end, N, shape->L, shape->G, shape->w, d, scale, row_lse ? row_lse : lse, score);
+  } else {
+    const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(q_win);
+    const __nv_bfloat16* kk = static_cast<const __nv_bfloat16*>(k);
+    if (!row_lse) {
+      if ((rc = set_smem(kvc::score_stats_simt<__nv_bfloat16>, sm1, "kvc_score")) != KVC_OK) return rc;
+      kvc::score_stats_simt<__nv_bfloat16><<<grid, kvc::SIMT_THREADS, sm1, stream>>>(
+          q, kk, chunk_end, N, shape->L, shape->G, shape->w, d, scale, part);
+      kvc::score_lse_merge<<<S, 256, 0, stream>>>(part, nblk, R, lse);
+    }
+    if ((rc = set_smem(kvc::score_colsum_simt<__nv_bfloat16>, sm2, "kvc_score")) != KVC_OK) return rc;
+    kvc::score_colsum_simt<__nv_bfloat16><<<grid, kvc::SIMT_THREADS, sm2, stream>>>(
+        q, kk, chunk_end, N, shape->L, shape->G, shape->w, d, scale, row_lse ? row_lse : lse, score);
+  }
+  return check_launch("kvc_score");
+}
+
+kvc_status kvc_select(const kvc_shape* shape, const float* score, const int8_t* policy, const int32_t* budget,
+                      float mass, const uint8_t* special_mask, const int32_t* chunk_end, int32_t C, int32_t* idx,
+                      int32_t max_sel, int32_t* count, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!policy || !budget || !count) return fail(KVC_ERR_INVALID_ARG, "kvc_select: policy, budget, count must be non-NULL");
+  if (max_sel < 0) return fail(KVC_ERR_SHAPE, "kvc_select: max_sel < 0");
+  if (!(mass > 0.f && mass <= 1.f)) return fail(KVC_ERR_INVALID_ARG, "kvc_select: mass %g not in (0, 1]", mass);
+  if (chunk_end && (C <= 0 || C > shape->L)) return fail(KVC_ERR_SHAPE, "kvc_select: C = %d not in [1, L]", C);
+  // The policy array is on the device; the kernel reads it. Pointers a policy may
+  // need are checked for presence here; a slot whose policy needs a missing
+  // pointer would read NULL, so the caller states which kinds occur via the pointers.
+  kvc::SelectParams p{};
+  p.score = score;
+  p.policy = policy;
+  p.budget = budget;
+  p.mass = mass;
+  p.special_mask = special_mask;
+  p.chunk_end = chunk_end;
+  p.C = chunk_end ? C : 0;
+  p.L = shape->L;
+  p.n_kv_heads = shape->n_kv_heads;
+  p.batch = shape->batch;
+  p.idx = idx;
+  p.max_sel = max_sel;
+  p.count = count;
+  p.key_cap = kvc::select_key_cap(shape->L, chunk_end ? C : 0);
+  const size_t smem = kvc::select_smem_bytes(p.key_cap);
+  if ((rc = set_smem(kvc::select_kernel, smem, "kvc_select")) != KVC_OK) return rc;
+  kvc::select_kernel<<<shape->n_slots, kvc::SEL_THREADS, smem, stream>>>(p);
+  count_launches(1);
+  return check_launch("kvc_select");
+}
+
+kvc_status kvc_alloc_budgets(const int32_t* counts, int32_t n_layers, int32_t spl, int32_t L, int32_t avg_B,
+                             int32_t floor_B, int32_t* budgets, int32_t* slot_budgets, cudaStream_t stream) {
+  if (!counts || !budgets) return fail(KVC_ERR_INVALID_ARG, "kvc_alloc_budgets: counts and budgets must be non-NULL");
+  if (n_layers <= 0 || n_layers > 1024 || spl <= 0 || L <= 0)
+    return fail(KVC_ERR_SHAPE, "kvc_alloc_budgets: need 1 <= n_layers <= 1024, spl >= 1, L >= 1");
+  if (!(0 <= floor_B && floor_B <= avg_B && avg_B <= L))
+    return fail(KVC_ERR_SHAPE, "kvc_alloc_budgets: need 0 <= floor_B (%d) <= avg_B (%d) <= L (%d)", floor_B, avg_B, L);
+  kvc::alloc_kernel<<<1, 1024, 0, stream>>>(counts, n_layers, spl, L, avg_B, floor_B, budgets, slot_budgets);
+  count_launches(1);
+  return check_launch("kvc_alloc_budgets");
+}
+
+kvc_status kvc_layout(const int32_t* count, int32_t n_slots, int32_t reserve, int64_t* off, int32_t* cap,
+                      cudaStream_t stream) {
+  if (!count || !off || !cap) return fail(KVC_ERR_INVALID_ARG, "kvc_layout: count, off, cap must be non-NULL");
+  if (n_slots <= 0 || reserve < 0) return fail(KVC_ERR_SHAPE, "kvc_layout: n_slots > 0 and reserve >= 0 required");
+  kvc::layout_kernel<<<1, 1024, 0, stream>>>(count, n_slots, reserve, off, cap);
+  count_launches(1);
+  return check_launch("kvc_layout");
+}
+
+kvc_status kvc_compact(const kvc_shape* shape, const void* k, const void* v, const int32_t* idx, int32_t max_sel,
+                       const int32_t* count, const int64_t* off, void* kp, void* vp, int64_t kp_rows, int32_t* len,
+                       cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!k || !v || !idx || !count || !off || !kp || !vp || !len)
+    return fail(KVC_ERR_INVALID_ARG, "kvc_compact: NULL pointer argument");
+  if (max_sel <= 0 || kp_rows < 0) return fail(KVC_ERR_SHAPE, "kvc_compact: max_sel > 0, kp_rows >= 0 required");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kp) || !aligned16(vp))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_compact: k, v, kp, vp must be 16-byte aligned");
+  DevInfo* di = nullptr;
+  if ((rc = dev_info(&di)) != KVC_OK) return rc;
+  const int tpr = (int)(shape->d * esize(shape->dtype) / 16);
+  const int blocks = di->sms * 8;
+  const uint4* k4 = static_cast<const uint4*>(k);
+  const uint4* v4 = static_cast<const uint4*>(v);
+  uint4* kp4 = static_cast<uint4*>(kp);
+  uint4* vp4 = static_cast<uint4*>(vp);
+  switch (tpr) {
+    case 8: kvc::compact_kernel<8, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, shape->n_slots,
+                                                                   shape->L, kp4, vp4, kp_rows, len); break;
+    case 16: kvc::compact_kernel<16, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, shape->n_slots,
+                                                                     shape->L, kp4, vp4, kp_rows, len); break;
+    case 32: kvc::compact_kernel<32, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, shape->n_slots,
+                                                                     shape->L, kp4, vp4, kp_rows, len); break;
+    default: return fail(KVC_ERR_UNSUPPORTED, "kvc_compact: row of %d bytes", tpr * 16);
+  }
+  count_launches(1);
+  return check_launch("kvc_compact");
+}
+
+kvc_status kvc_append(const kvc_shape* shape, const void* k_new, const void* v_new, const int64_t* off,
+                      const int32_t* cap, int32_t* len, void* kp, void* vp, int64_t kp_rows, cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!k_new || !v_new || !off || !cap || !len || !kp || !vp)
+    return fail(KVC_ERR_INVALID_ARG, "kvc_append: NULL pointer argument");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kp) || !aligned16(vp))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_append: buffers must be 16-byte aligned");
+  const int tpr = (int)(shape->d * esize(shape->dtype) / 16);
+  kvc::append_kernel<<<shape->n_slots, tpr, 0, stream>>>(static_cast<const uint4*>(k_new),
+                                                          static_cast<const uint4*>(v_new), off, cap, len,
+                                                          static_cast<uint4*>(kp), static_cast<uint4*>(vp), kp_rows,
+                                                          tpr);
+  count_launches(1);
+  return check_launch("kvc_append");
+}
+
+kvc_status kvc_decode_attn(const kvc_shape* shape, const void* q, const void* kp, const void* vp, const int64_t* off,
+                           const int32_t* len, int64_t kp_rows, float* out, void* ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!q || !kp || !vp || !off || !len || !out) return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn: NULL pointer argument");
+  if (shape->n_slots > kvc::DEC_MAX_SLOTS)
+    return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: %d slots > %d", shape->n_slots, kvc::DEC_MAX_SLOTS);
+  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(ws))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn: q, kp, vp, ws must be 16-byte aligned");
+  DevInfo* di = nullptr;
+  if ((rc = dev_info(&di)) != KVC_OK) return rc;
+  const DecodeWs w = decode_ws_layout(shape, di->sms);
+  if (!ws || ws_bytes < w.total)
+    return fail(KVC_ERR_WORKSPACE, "kvc_decode_attn: workspace %zu B < required %zu B", ws_bytes, w.total);
+  unsigned char* wsb = static_cast<unsigned char*>(ws);
+  kvc::DecodeParams p{};
+  p.q = q;
+  p.kp = kp;
+  p.vp = vp;
+  p.off = off;
+  p.len = len;
+  p.kp_rows = kp_rows;
+  p.S = shape->n_slots;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)shape->d);
+  p.out = out;
+  p.partial = reinterpret_cast<float*>(wsb + w.part_off);
+  p.counters = reinterpret_cast<int*>(wsb + w.cnt_off);
+  if (shape->dtype == KVC_BF16) {
+    if (shape->d == 128) return decode_by_g<__nv_bfloat16, 128>(shape->G, p, di->sms, stream);
+    return decode_by_g<__nv_bfloat16, 64>(shape->G, p, di->sms, stream);
+  }
+  if (shape->d == 128) return decode_by_g<float, 128>(shape->G, p, di->sms, stream);
+  return decode_by_g<float, 64>(shape->G, p, di->sms, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,126 @@
+"""One workload through the C ABI: window scoring -> selection (-> ZigZagKV
+allocation) -> layout -> compaction, then per decode step append -> decode.
+
+Host-side orchestration only: buffers are torch CUDA tensors allocated once,
+every step is a libkvc call on one stream.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (kvc_score, kvc_select, kvc_alloc_budgets, kvc_layout, kvc_compact, kvc_append, kvc_decode_attn,
+               kvc_workspace_size, make_shape, KVC_WS_SCORE, KVC_WS_DECODE, KVC_POL_TOPB, KVC_POL_MASS_COUNT,
+               KVC_POL_CHUNK)
+
+
+def _round16(x: int) -> int:
+    return (x + 15) // 16 * 16
+
+
+class KvcPipeline:
+    """Buffers and call sequence for one workload (see workloads.configs).
+
+    `inp` is a workloads.Inputs whose tensors are on the target CUDA device.
+    """
+
+    def __init__(self, wl, inp, device=None):
+        self.wl = wl
+        self.inp = inp
+        dev = torch.device(device) if device is not None else inp.k.device
+        self.dev = dev
+        S, G, d, L = wl.n_slots, wl.G, wl.d, wl.L
+        dt = inp.k.dtype
+        self.shape = make_shape(S, G, d, L, wl.w, wl.hkv, wl.batch, dt)
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.chunk_end = inp.chunk_end
+        self.C = int(inp.chunk_end.numel()) if inp.chunk_end is not None else 0
+        if wl.w > 0:
+            N = self.C if wl.policy == "chunk" else L
+            self.score = torch.empty((S, N), dtype=torch.float32, device=dev)
+            self.ws_score = torch.zeros(kvc_workspace_size(KVC_WS_SCORE, self.shape, self.C), dtype=torch.uint8,
+                                        device=dev)
+        else:
+            self.score = None
+        self.max_sel = min(wl.top_b, L) if wl.policy == "topb" else L
+        self.idx = torch.empty((S, self.max_sel), **i32)
+        self.count = torch.empty((S,), **i32)
+        self.budget = torch.empty((S,), **i32)
+        self.policy = torch.empty((S,), dtype=torch.int8, device=dev)
+        if wl.policy == "topb":
+            self.policy.fill_(KVC_POL_TOPB)
+            self.budget.fill_(wl.top_b)
+        elif wl.policy == "zigzag":
+            self.mass_count = torch.empty((S,), **i32)
+            self.layer_budget = torch.empty((wl.n_layers,), **i32)
+            self.pol_mass = torch.full((S,), KVC_POL_MASS_COUNT, dtype=torch.int8, device=dev)
+            self.policy.fill_(KVC_POL_TOPB)
+        elif wl.policy == "fastgen":
+            self.policy.copy_(inp.policy)
+            self.budget.fill_(wl.local_window)
+        elif wl.policy == "chunk":
+            self.policy.fill_(KVC_POL_CHUNK)
+            self.budget.fill_(wl.chunk_target)
+        self.off = torch.empty((S + 1,), dtype=torch.int64, device=dev)
+        self.cap = torch.empty((S,), **i32)
+        self.len = torch.empty((S,), **i32)
+        self.kp_rows = S * _round16(self.max_sel + wl.reserve)
+        self.kp = torch.empty((self.kp_rows, d), dtype=dt, device=dev)
+        self.vp = torch.empty((self.kp_rows, d), dtype=dt, device=dev)
+        self.out = torch.empty((S * G, d), dtype=torch.float32, device=dev)
+        self.ws_decode = torch.zeros(kvc_workspace_size(KVC_WS_DECODE, self.shape), dtype=torch.uint8, device=dev)
+
+    # ---- the hot path
+    def score_step(self, stream=None):
+        wl, inp = self.wl, self.inp
+        if wl.policy == "chunk":
+            kvc_score(self.shape, inp.q_win, inp.k, self.score, self.ws_score, chunk_end=self.chunk_end, C=self.C,
+                      stream=stream)
+        elif wl.w > 0:
+            kvc_score(self.shape, inp.q_win, inp.k, self.score, self.ws_score, stream=stream)
+
+    def select_step(self, stream=None):
+        wl, inp = self.wl, self.inp
+        if wl.policy == "zigzag":
+            kvc_select(self.shape, self.score, self.pol_mass, self.budget, None, self.mass_count, mass=wl.mass,
+                       stream=stream)
+            kvc_alloc_budgets(self.mass_count, wl.n_layers, wl.slots_per_layer, wl.L, wl.avg_budget,
+                              wl.floor_budget, self.layer_budget, self.budget, stream=stream)
+            kvc_select(self.shape, self.score, self.policy, self.budget, self.idx, self.count, stream=stream)
+        elif wl.policy == "fastgen":
+            kvc_select(self.shape, None, self.policy, self.budget, self.idx, self.count,
+                       special_mask=inp.special_mask, stream=stream)
+        elif wl.policy == "chunk":
+            kvc_select(self.shape, self.score, self.policy, self.budget, self.idx, self.count,
+                       chunk_end=self.chunk_end, C=self.C, stream=stream)
+        else:
+            kvc_select(self.shape, self.score, self.policy, self.budget, self.idx, self.count, stream=stream)
+
+    def compact_step(self, stream=None):
+        kvc_layout(self.count, self.wl.reserve, self.off, self.cap, stream=stream)
+        kvc_compact(self.shape, self.inp.k, self.inp.v, self.idx, self.count, self.off, self.kp, self.vp, self.len,
+                    stream=stream)
+
+    def compress(self, stream=None):
+        self.score_step(stream)
+        self.select_step(stream)
+        self.compact_step(stream)
+
+    def decode_step(self, t: int, q=None, k_new=None, v_new=None, out=None, stream=None):
+        inp = self.inp
+        q = inp.q_dec[t] if q is None else q
+        k_new = inp.k_dec[t] if k_new is None else k_new
+        v_new = inp.v_dec[t] if v_new is None else v_new
+        out = self.out if out is None else out
+        kvc_append(self.shape, k_new, v_new, self.off, self.cap, self.len, self.kp, self.vp, stream=stream)
+        kvc_decode_attn(self.shape, q, self.kp, self.vp, self.off, self.len, out, self.ws_decode, stream=stream)
+        return out
+
+    def run(self, steps=None, record=False, stream=None):
+        self.compress(stream)
+        outs = []
+        n = self.wl.steps if steps is None else steps
+        for t in range(n):
+            o = self.decode_step(t, stream=stream)
+            if record:
+                outs.append(o.clone())
+        return outs

@@ -1,0 +1,314 @@
+"""CUDA path vs the fp64 oracle, through the C ABI, on the same seeded inputs.
+
+Small workloads are checked on every slot and step; the full-size workloads run
+in the same launch configuration the benchmark times and are checked on sampled
+slots and steps (the oracle computes them one by one)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from workloads import get, make_inputs, POL_LOCAL, POL_SPECIAL, POL_FULL
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import sparse_decode_attention_window_b200 as kvc
+    kvc.library()
+    yield
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def run_and_check(wl, slots=None, steps=None, gen_device="cpu", check_scores=True):
+    """Run the workload through the ABI and check it against the oracle.
+    slots: slots to check (default all); steps: decode steps to check (default all)."""
+    from sparse_decode_attention_window_b200.pipeline import KvcPipeline
+    import sparse_decode_attention_window_b200 as kvc
+
+    if gen_device == "cpu":
+        from dataclasses import replace
+        inp_host = make_inputs(wl, "cpu")
+        inp = replace(inp_host, **{f: (getattr(inp_host, f).cuda() if getattr(inp_host, f) is not None else None)
+                                   for f in ("q_win", "k", "v", "q_dec", "k_dec", "v_dec", "policy",
+                                             "special_mask", "chunk_end")})
+    else:
+        inp = inp_host = make_inputs(wl, "cuda")
+    S, G, L, d = wl.n_slots, wl.G, wl.L, wl.d
+    slots = list(range(S)) if slots is None else list(slots)
+    steps = list(range(wl.steps)) if steps is None else list(steps)
+
+    pipe = KvcPipeline(wl, inp)
+    pipe.compress()
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    count = _np(pipe.count).astype(np.int64)
+    idx = _np(pipe.idx)
+    off, cap, ln = _np(pipe.off), _np(pipe.cap), _np(pipe.len)
+
+    # layout: exact given the GPU counts
+    ref_off, ref_cap = O.layout(count, wl.reserve)
+    np.testing.assert_array_equal(off, ref_off)
+    np.testing.assert_array_equal(cap, ref_cap)
+    np.testing.assert_array_equal(ln, count)
+
+    k_cpu = lambda s: inp.k[s].cpu()
+    qw_cpu = lambda s: inp.q_win[s * G:(s + 1) * G].cpu()
+    ce = _np(inp.chunk_end) if inp.chunk_end is not None else None
+    sc_gpu = _np(pipe.score) if pipe.score is not None else None
+
+    ref_scores = {}
+    if wl.w > 0:
+        for s in slots:
+            if wl.policy == "chunk":
+                ref_scores[s] = O.chunk_scores(qw_cpu(s), k_cpu(s)[None], L, ce)[0]
+            else:
+                ref_scores[s] = O.window_scores(qw_cpu(s), k_cpu(s)[None], L)[0]
+            if check_scores:
+                P.check_scores(sc_gpu[s], ref_scores[s], wl.dtype, f"score slot {s}")
+
+    if wl.policy == "zigzag":
+        mc = _np(pipe.mass_count).astype(np.int64)
+        for s in slots:
+            P.check_mass_count(int(mc[s]), ref_scores[s], wl.mass, f"LMBA slot {s}")
+        ref_budget = O.allocate_budgets(mc.reshape(wl.n_layers, wl.slots_per_layer), L, wl.avg_budget,
+                                        wl.floor_budget)
+        np.testing.assert_array_equal(_np(pipe.layer_budget), ref_budget)
+        np.testing.assert_array_equal(_np(pipe.budget), np.repeat(ref_budget, wl.slots_per_layer))
+
+    for s in slots:
+        got = idx[s, :count[s]].astype(np.int64)
+        if wl.policy == "topb":
+            P.check_topb(got, ref_scores[s], wl.top_b, f"top-B slot {s}")
+        elif wl.policy == "zigzag":
+            P.check_topb(got, ref_scores[s], int(_np(pipe.layer_budget)[s // wl.slots_per_layer]), f"slot {s}")
+        elif wl.policy == "fastgen":
+            pol = int(inp_host.policy[s])
+            b = (s // wl.hkv) % wl.batch
+            if pol == POL_LOCAL:
+                want = O.local_indices(L, wl.local_window)
+            elif pol == POL_SPECIAL:
+                want = O.special_indices(_np(inp.special_mask[b]))
+            else:
+                want = O.full_indices(L)
+            np.testing.assert_array_equal(got, want, err_msg=f"policy slot {s}")
+        elif wl.policy == "chunk":
+            P.check_chunks(got, ref_scores[s], ce, wl.chunk_target, f"chunks slot {s}")
+        # packed rows are the kept rows, bit for bit
+        o, n = int(off[s]), int(count[s])
+        gi = torch.from_numpy(got).to(inp.k.device)
+        assert torch.equal(pipe.kp[o:o + n], inp.k[s].index_select(0, gi)), f"packed K slot {s}"
+        assert torch.equal(pipe.vp[o:o + n], inp.v[s].index_select(0, gi)), f"packed V slot {s}"
+
+    # decode: the oracle attends over the GPU's (checked) selection plus the appended tokens
+    worst = 0.0
+    want_steps = set(steps)
+    outs = {}
+    for t in range(max(steps) + 1 if steps else 0):
+        o_t = pipe.decode_step(t)
+        if t in want_steps:
+            outs[t] = _np(o_t).copy()
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    for s in slots:
+        sel = idx[s, :count[s]].astype(np.int64)
+        ks = O._f64(inp.k[s].cpu())[sel]
+        vs = O._f64(inp.v[s].cpu())[sel]
+        kn = O._f64(inp.k_dec[:, s].cpu())
+        vn = O._f64(inp.v_dec[:, s].cpu())
+        for t in sorted(want_steps):
+            keys = np.concatenate([ks, kn[:t + 1]])
+            vals = np.concatenate([vs, vn[:t + 1]])
+            n = keys.shape[0]
+            q = O._f64(inp.q_dec[t, s * G:(s + 1) * G].cpu())
+            ref = O.decode_attention(q, keys, vals, [0, n], [n], G)
+            worst = max(worst, P.check_out(outs[t][s * G:(s + 1) * G], ref, wl.dtype, f"decode slot {s} step {t}"))
+    return pipe, worst
+
+
+# ---------------------------------------------------------------- the workloads, small
+def test_tiny_workload_all_slots_all_steps():
+    run_and_check(get("tiny"))
+
+
+@pytest.mark.parametrize("L,top_b", [(1024, 128), (1000, 64)])
+def test_llama8b_shape_small_context(L, top_b):
+    run_and_check(get("llama8b").scaled(batch=2, L=L, top_b=top_b, steps=6))
+
+
+def test_zigzag_small():
+    run_and_check(get("zigzag").scaled(n_layers=4, L=2048, steps=5))
+
+
+def test_fastgen_small():
+    run_and_check(get("fastgen").scaled(batch=2, L=3000, steps=7))
+
+
+def test_chunk_small():
+    run_and_check(get("chunk").scaled(L=6000, steps=5))
+
+
+# ---------------------------------------------------------------- full sizes (benchmark launch configuration)
+def test_llama8b_full_size():
+    wl = get("llama8b")
+    run_and_check(wl, slots=range(wl.n_slots), steps=[0, 31, 63], gen_device="cuda")
+
+
+def test_zigzag_full_size_sampled():
+    wl = get("zigzag")
+    rng = np.random.default_rng(0)
+    slots = sorted(rng.choice(wl.n_slots, size=12, replace=False).tolist())
+    run_and_check(wl, slots=slots, steps=[0, 31], gen_device="cuda")
+
+
+def test_fastgen_full_size_sampled():
+    wl = get("fastgen")
+    run_and_check(wl, slots=[0, 5, 17, 33, 50, 63], steps=[0, 127], gen_device="cuda")
+
+
+def test_chunk_full_size_sampled():
+    wl = get("chunk")
+    run_and_check(wl, slots=[0, 3, 7], steps=[0, 255], gen_device="cuda")
+
+
+# ---------------------------------------------------------------- edge cases
+@pytest.mark.parametrize("L", [1, 7, 255, 256, 257, 4099])
+def test_ragged_context_lengths(L):
+    w = min(4, L)
+    run_and_check(get("llama8b").scaled(batch=1, hq=8, hkv=2, L=L, w=w, top_b=max(1, L // 3), steps=2))
+
+
+@pytest.mark.parametrize("hq,hkv", [(2, 2), (4, 2), (8, 2)])
+def test_gqa_group_sizes(hq, hkv):
+    run_and_check(get("llama8b").scaled(batch=1, hq=hq, hkv=hkv, L=600, w=8, top_b=100, steps=3))
+
+
+@pytest.mark.parametrize("d,dtype", [(64, "bf16"), (128, "fp32")])
+def test_head_dims_and_dtypes(d, dtype):
+    run_and_check(get("llama8b").scaled(batch=1, d=d, dtype=dtype, L=700, w=16, top_b=90, steps=3))
+
+
+def test_window_of_one():
+    run_and_check(get("llama8b").scaled(batch=1, L=513, w=1, top_b=50, steps=2))
+
+
+@pytest.mark.parametrize("top_b", [1, 511, 512, 100000])
+def test_budget_extremes(top_b):
+    run_and_check(get("llama8b").scaled(batch=1, L=512, w=8, top_b=top_b, steps=2))
+
+
+def test_mass_count_closed_forms_on_gpu():
+    """Uniform scores keep ceil(0.9 L); a one-hot distribution keeps one token."""
+    import sparse_decode_attention_window_b200 as kvc
+    L = 1000
+    sh = kvc.make_shape(3, 1, 64, L, 1, 3, 1, torch.bfloat16)
+    sc = torch.zeros((3, L), dtype=torch.float32, device="cuda")
+    sc[0] = 1.0
+    sc[1, 123] = 5.0
+    sc[2] = torch.linspace(1.0, 2.0, L, device="cuda")
+    pol = torch.full((3,), kvc.KVC_POL_MASS_COUNT, dtype=torch.int8, device="cuda")
+    bud = torch.zeros(3, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(3, dtype=torch.int32, device="cuda")
+    kvc.kvc_select(sh, sc, pol, bud, None, cnt, mass=0.9)
+    c = cnt.cpu().numpy()
+    assert c[0] == 900 and c[1] == 1
+    P.check_mass_count(int(c[2]), _np(sc[2]).astype(np.float64))
+
+
+def test_empty_slot_decodes_to_zero_and_append_overflow_is_reported():
+    import sparse_decode_attention_window_b200 as kvc
+    S, G, d = 3, 2, 64
+    sh = kvc.make_shape(S, G, d, 16, 0, S, 1, torch.bfloat16)
+    count = torch.tensor([0, 5, 0], dtype=torch.int32, device="cuda")
+    off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    cap = torch.empty(S, dtype=torch.int32, device="cuda")
+    kvc.kvc_layout(count, 0, off, cap)
+    assert cap.cpu().tolist() == [0, 16, 0]
+    rows = int(off[-1])
+    kp = torch.randn(rows, d, device="cuda").to(torch.bfloat16)
+    vp = torch.randn(rows, d, device="cuda").to(torch.bfloat16)
+    ln = count.clone()
+    q = torch.randn(S * G, d, device="cuda").to(torch.bfloat16)
+    out = torch.full((S * G, d), 7.0, device="cuda")
+    ws = torch.zeros(kvc.kvc_workspace_size(kvc.KVC_WS_DECODE, sh), dtype=torch.uint8, device="cuda")
+    kvc.kvc_decode_attn(sh, q, kp, vp, off, ln, out, ws)
+    o = _np(out)
+    assert (o[0:2] == 0).all() and (o[4:6] == 0).all()
+    ref = O.decode_attention(q[2:4].cpu(), kp[:5].cpu(), vp[:5].cpu(), [0, 5], [5], G)
+    P.check_out(o[2:4], ref, "bf16")
+    # slot 0 and 2 have capacity 0: appending overflows there (reported, not faulted)
+    kn = torch.randn(S, d, device="cuda").to(torch.bfloat16)
+    kvc.kvc_append(sh, kn, kn, off, cap, ln, kp, vp)
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.kvc_get_status()
+    assert e.value.status == 7 and "append-overflow" in str(e.value)
+    assert ln.cpu().tolist() == [0, 6, 0]
+    kvc.kvc_get_status()   # the word was cleared
+
+
+def test_special_policy_with_no_special_tokens():
+    import sparse_decode_attention_window_b200 as kvc
+    L = 300
+    sh = kvc.make_shape(2, 1, 64, L, 0, 2, 1, torch.bfloat16)
+    mask = torch.zeros((1, L), dtype=torch.uint8, device="cuda")
+    pol = torch.full((2,), kvc.KVC_POL_SPECIAL, dtype=torch.int8, device="cuda")
+    bud = torch.zeros(2, dtype=torch.int32, device="cuda")
+    idx = torch.full((2, L), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(2, dtype=torch.int32, device="cuda")
+    kvc.kvc_select(sh, None, pol, bud, idx, cnt, special_mask=mask)
+    assert cnt.cpu().tolist() == [0, 0]
+
+
+def test_decode_is_independent_of_how_tokens_split_over_ctas():
+    """The same slot decoded alone and next to other slots (different CTA ranges) agrees."""
+    import sparse_decode_attention_window_b200 as kvc
+    d, G = 128, 4
+    torch.manual_seed(0)
+    lens = [5000, 3, 777, 12000]
+    S = len(lens)
+    sh = kvc.make_shape(S, G, d, 16384, 0, S, 1, torch.bfloat16)
+    count = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    cap = torch.empty(S, dtype=torch.int32, device="cuda")
+    kvc.kvc_layout(count, 0, off, cap)
+    rows = int(off[-1])
+    kp = torch.randn(rows, d, device="cuda").to(torch.bfloat16)
+    vp = torch.randn(rows, d, device="cuda").to(torch.bfloat16)
+    q = torch.randn(S * G, d, device="cuda").to(torch.bfloat16)
+    out = torch.empty((S * G, d), device="cuda")
+    ws = torch.zeros(kvc.kvc_workspace_size(kvc.KVC_WS_DECODE, sh), dtype=torch.uint8, device="cuda")
+    kvc.kvc_decode_attn(sh, q, kp, vp, off, count, out, ws)
+    sh1 = kvc.make_shape(1, G, d, 16384, 0, 1, 1, torch.bfloat16)
+    for s in range(S):
+        o1 = torch.empty((G, d), device="cuda")
+        o_s = int(off[s])
+        off1 = torch.tensor([0, int(cap[s])], dtype=torch.int64, device="cuda")
+        kvc.kvc_decode_attn(sh1, q[s * G:(s + 1) * G].contiguous(), kp[o_s:].contiguous(), vp[o_s:].contiguous(),
+                            off1, count[s:s + 1].clone(), o1, ws)
+        P.check_out(_np(o1), _np(out[s * G:(s + 1) * G]).astype(np.float64), "bf16", f"slot {s}")
+        ref = O.decode_attention(q[s * G:(s + 1) * G].cpu(), kp[o_s:o_s + lens[s]].cpu(), vp[o_s:o_s + lens[s]].cpu(),
+                                 [0, lens[s]], [lens[s]], G)
+        P.check_out(_np(out[s * G:(s + 1) * G]), ref, "bf16", f"slot {s} vs oracle")
+
+
+def test_wide_window_takes_cuda_core_scoring_path():
+    """G*w = 256 rows exceeds the tensor-core tile: scoring runs on the CUDA-core kernels."""
+    run_and_check(get("llama8b").scaled(batch=1, hq=16, hkv=2, L=900, w=32, top_b=100, steps=0), steps=[])
+
+
+def test_cuda_core_scoring_path_on_bf16_workloads():
+    """The CUDA-core scoring kernels, forced for bf16, pass the same oracle checks."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, KVC_SCORE_PATH="simt")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        "-k", "llama8b_shape_small_context or zigzag_small or chunk_small"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
