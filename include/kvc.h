@@ -203,6 +203,26 @@ kvc_status kvc_decode_attn(const kvc_shape* shape, const void* q, const void* kp
                            int64_t kp_rows, float* out, void* ws, size_t ws_bytes,
                            cudaStream_t stream);
 
+/*
+ * kvc_decode_attn_noalloc - kvc_decode_attn for callers that cannot allocate
+ *   device memory: code that runs inside a runtime owning every device buffer
+ *   (a plugin or operator that is handed only its inputs and outputs at enqueue
+ *   time, with no allocator and no workspace handle), or loops where a
+ *   cudaMalloc's implicit device synchronisation is not acceptable. The paper has
+ *   no counterpart; this is a property of the library, not of the method.
+ *   Same arguments and results as kvc_decode_attn minus the workspace: the
+ *   scratch lives in a fixed 4 MiB array inside the library (held by every GPU
+ *   that loads it, until exit). The first call on each device looks up that
+ *   array's device address (make it before any stream capture). Shapes whose
+ *   scratch (kvc_workspace_size(KVC_WS_DECODE, ...)) exceeds 4 MiB are rejected
+ *   with KVC_ERR_WORKSPACE. All calls share the array and each call clears the
+ *   part that must start at zero: calls that overlap on the GPU (for example on
+ *   two streams) race and must not be issued.
+ */
+kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const void* kp,
+                                   const void* vp, const int64_t* off, const int32_t* len,
+                                   int64_t kp_rows, float* out, cudaStream_t stream);
+
 /* Bytes of workspace the call `which` (KVC_WS_*) needs for this shape (C: chunks, 0 if none). */
 size_t kvc_workspace_size(int which, const kvc_shape* shape, int32_t C);
 

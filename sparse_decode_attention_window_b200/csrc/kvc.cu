@@ -185,6 +185,39 @@ kvc_status decode_by_g(int G, const kvc::DecodeParams& p, int sms, cudaStream_t 
 
 }  // namespace
 
+// ---- scratch for kvc_decode_attn_noalloc
+// Fixed device-side scratch for callers that cannot allocate device memory. Every
+// GPU that loads this library holds these bytes until the process exits. In host
+// code `g_noalloc_scratch` is only a stand-in for the symbol, never a device
+// address: the address is fetched per device with cudaGetSymbolAddress below.
+#define KVC_NOALLOC_SCRATCH_BYTES (4u << 20)
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KVC_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices];
+cudaError_t g_noalloc_rc[kMaxDevices];
+std::once_flag g_noalloc_once[kMaxDevices];
+
+// Device address of the scratch array on the current device, looked up once per
+// device (the first call on a device does this; make that call before any stream
+// capture, since the lookup may load the module).
+kvc_status noalloc_scratch(unsigned char** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(KVC_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::call_once(g_noalloc_once[dev], [dev] {
+    void* p = nullptr;
+    g_noalloc_rc[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    g_noalloc_ptr[dev] = p;
+  });
+  if (g_noalloc_rc[dev] != cudaSuccess || !g_noalloc_ptr[dev])
+    return fail(KVC_ERR_CUDA, "scratch address on device %d: %s", dev, cudaGetErrorString(g_noalloc_rc[dev]));
+  *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
+  return KVC_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char* kvc_last_error(void) { return g_last_error.c_str(); }
@@ -412,6 +445,52 @@ kvc_status kvc_decode_attn(const kvc_shape* shape, const void* q, const void* kp
   if (!ws || ws_bytes < w.total)
     return fail(KVC_ERR_WORKSPACE, "kvc_decode_attn: workspace %zu B < required %zu B", ws_bytes, w.total);
   unsigned char* wsb = static_cast<unsigned char*>(ws);
+  kvc::DecodeParams p{};
+  p.q = q;
+  p.kp = kp;
+  p.vp = vp;
+  p.off = off;
+  p.len = len;
+  p.kp_rows = kp_rows;
+  p.S = shape->n_slots;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)shape->d);
+  p.out = out;
+  p.partial = reinterpret_cast<float*>(wsb + w.part_off);
+  p.counters = reinterpret_cast<int*>(wsb + w.cnt_off);
+  if (shape->dtype == KVC_BF16) {
+    if (shape->d == 128) return decode_by_g<__nv_bfloat16, 128>(shape->G, p, di->sms, stream);
+    return decode_by_g<__nv_bfloat16, 64>(shape->G, p, di->sms, stream);
+  }
+  if (shape->d == 128) return decode_by_g<float, 128>(shape->G, p, di->sms, stream);
+  return decode_by_g<float, 64>(shape->G, p, di->sms, stream);
+}
+
+// Decode attention without a caller workspace: same kernel and results as
+// kvc_decode_attn, with its scratch in the fixed array above. Allocates nothing.
+kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const void* kp, const void* vp,
+                                   const int64_t* off, const int32_t* len, int64_t kp_rows, float* out,
+                                   cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!q || !kp || !vp || !off || !len || !out)
+    return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn_noalloc: NULL pointer argument");
+  if (shape->n_slots > kvc::DEC_MAX_SLOTS)
+    return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn_noalloc: %d slots > %d", shape->n_slots, kvc::DEC_MAX_SLOTS);
+  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn_noalloc: q, kp, vp must be 16-byte aligned");
+  DevInfo* di = nullptr;
+  if ((rc = dev_info(&di)) != KVC_OK) return rc;
+  const DecodeWs w = decode_ws_layout(shape, di->sms);
+  if (w.total > KVC_NOALLOC_SCRATCH_BYTES)
+    return fail(KVC_ERR_WORKSPACE,
+                "kvc_decode_attn_noalloc: this shape needs %zu B of scratch; the fixed array holds %u B "
+                "(use kvc_decode_attn with a workspace)",
+                w.total, (unsigned)KVC_NOALLOC_SCRATCH_BYTES);
+  unsigned char* wsb = nullptr;
+  if ((rc = noalloc_scratch(&wsb)) != KVC_OK) return rc;
+  // the merge tickets must start at zero; the array keeps whatever the last call left
+  cudaError_t e = cudaMemsetAsync(wsb + w.cnt_off, 0, w.cnt_bytes, stream);
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "kvc_decode_attn_noalloc: clear: %s", cudaGetErrorString(e));
   kvc::DecodeParams p{};
   p.q = q;
   p.kp = kp;
