@@ -50,77 +50,82 @@ def esize(wl):
     return 4 if wl.dtype == "fp32" else 2
 
 
-def work_per_step(wl, counts):
-    """Algorithmic bytes / flops of each phase of one step (no padding, no second scoring pass)."""
+def work_per_step(wl, counts, n_chunks=0):
+    """Algorithmic bytes / flops of each phase of one step (no padding, no second scoring pass).
+    Chunk scoring reads one key per chunk (plus the chunk ends)."""
     es = esize(wl)
     S, G, d, L, w = wl.n_slots, wl.G, wl.d, wl.L, wl.w
     out = {}
     if w > 0:
-        N = L
-        out["score_bytes"] = S * L * d * es + S * G * w * d * es + S * N * 4
-        out["score_flops"] = 2.0 * S * G * w * L * d
+        N = n_chunks if wl.policy == "chunk" else L
+        out["score_bytes"] = S * N * d * es + S * G * w * d * es + S * N * 4 + (N * 4 if n_chunks else 0)
+        out["score_flops"] = 2.0 * S * G * w * N * d
     kept = int(np.sum(counts))
     out["compact_bytes"] = kept * 2 * d * es * 2 + kept * 4
     dec = []
     for t in range(wl.steps):
         rows = kept + S * (t + 1)
-        dec.append(rows * 2 * d * es + S * G * d * es + S * G * d * 4)
+        # K and V of every cached row, q, the fp32 output, and the new token read + written
+        dec.append(rows * 2 * d * es + S * G * d * es + S * G * d * 4 + 2 * S * 2 * d * es)
     out["decode_bytes"] = dec
     return out
 
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons of this process's GPU, sampled every few ms by
+    NVML in a thread while the timed region runs (nvidia-smi as a fallback)."""
 
-    def __init__(self, device_index: int):
-        self.proc = None
-        self.path = None
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.004):
+        import threading
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.handle = None
         try:
+            import pynvml
+            pynvml.nvmlInit()
             p = torch.cuda.get_device_properties(device_index)
-            self.bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            bus = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.nvml = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
         except Exception:
-            self.bus = None
+            self.handle = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(self.period)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
-        if self.bus:
-            cmd += ["-i", self.bus]
-        try:
-            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        if self.handle is None:
+            return
+        import threading
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for nm, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(nm)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        self._stop.set()
+        self._thread.join(timeout=2)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, every 4 ms"}
 
 
 # ------------------------------------------------------------------ oracle timing (CPU baseline / reference arm)
@@ -209,7 +214,6 @@ def cuda_arm(args, wl, rank, world, local_rank):
     out_all = torch.empty((n_dec,) + tuple(pipe.out.shape), dtype=torch.float32, device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
     e = [ev() for _ in range(4)]
-    ea = [ev() for _ in range(n_dec)]
     ed = [ev() for _ in range(n_dec)]
 
     def step_calls():
@@ -222,10 +226,8 @@ def cuda_arm(args, wl, rank, world, local_rank):
         pipe.compact_step()
         e[3].record()
         for t in range(n_dec):
-            kvc.kvc_append(pipe.shape, inp.k_dec[t], inp.v_dec[t], pipe.off, pipe.cap, pipe.len, pipe.kp, pipe.vp)
-            ea[t].record()
-            kvc.kvc_decode_attn(pipe.shape, inp.q_dec[t], pipe.kp, pipe.vp, pipe.off, pipe.len, out_all[t],
-                                pipe.ws_decode)
+            # one launch per token step: append the new K/V rows and decode (kvc_append_decode)
+            pipe.decode_step(t, out=out_all[t])
             ed[t].record()
 
     # eager warm-up: loads every kernel and sets its attributes before capture
@@ -235,7 +237,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
     torch.cuda.synchronize()
     kvc.kvc_get_status()
     counts = pipe.count.cpu().numpy()
-    work = work_per_step(wl, counts)
+    work = work_per_step(wl, counts, pipe.C)
 
     # the whole step as one CUDA graph (launch-bound decode loop: 2 launches per token step)
     graph = torch.cuda.CUDAGraph()
@@ -256,7 +258,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
     clocks.start()
     barrier()
     torch.cuda.synchronize()
-    step_ms, score_ms, select_ms, compact_ms, dec_ms, app_ms = [], [], [], [], [], []
+    step_ms, score_ms, select_ms, compact_ms, dec_ms = [], [], [], [], []
     for _ in range(args.steps):
         flush.zero_()          # L2 flushed between steps, outside the timed events
         graph.replay()
@@ -267,8 +269,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
         step_ms.append(e[0].elapsed_time(ed[-1]))
         prev = e[3]
         for t in range(n_dec):
-            app_ms.append(prev.elapsed_time(ea[t]))
-            dec_ms.append(ea[t].elapsed_time(ed[t]))
+            dec_ms.append(prev.elapsed_time(ed[t]))
             prev = ed[t]
     torch.cuda.synchronize()
     barrier()
@@ -312,8 +313,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "score_us": 1000.0 * statistics.mean(score_ms),
         "select_us": 1000.0 * statistics.mean(select_ms),
         "compact_us": 1000.0 * statistics.mean(compact_ms),
-        "append_us_mean": 1000.0 * statistics.mean(app_ms),
-        "decode_us_mean": dec_us,
+        "append_decode_us_mean": dec_us,
     }
     if "score_bytes" in work:
         s_us = phases["score_us"]
@@ -330,11 +330,11 @@ def cuda_arm(args, wl, rank, world, local_rank):
                    "layers": wl.n_layers, "parallelism": f"replicas x{world}",
                    "l2": "flushed (2x L2 write) before every step, outside the timed events; "
                          "within a step the compacted cache is re-read by each decode step"},
-        "decode_tokens_per_s": wl.batch / ((statistics.mean(app_ms) + statistics.mean(dec_ms)) / 1000.0) * world,
+        "decode_tokens_per_s": wl.batch / (statistics.mean(dec_ms) / 1000.0) * world,
         "decode_hbm_gbs": dec_gbs,
         "score_select_compact_us_per_layer": ssc_us / wl.n_layers,
         "phases": phases,
-        "roofline": {"kernel": "kvc_decode_attn", "bound": "hbm", "achieved": dec_gbs, "peak": hbm,
+        "roofline": {"kernel": "decode_mma_kernel (kvc_append_decode)", "bound": "hbm", "achieved": dec_gbs, "peak": hbm,
                      "unit": "GB/s", "frac": dec_gbs / hbm, "traffic": None,
                      "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": dec_bytes},
         "clocks": clk,
@@ -380,7 +380,7 @@ def e2e_run(args, wl, inp, graph, out_all, dev):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama8b")
     ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])

@@ -11,6 +11,7 @@
  *   kvc_compact        gather of the kept rows into the packed per-head cache
  *   kvc_append         one new token per slot per decode step
  *   kvc_decode_attn    split-K GQA decode attention over the ragged packed cache
+ *   kvc_append_decode  the two above fused into one launch (the per-step call)
  *
  * Sources: "ZigZagKV: Dynamic KV Cache Compression for Long-context Modeling based
  * on Layer Uncertainty" (arXiv 2412.09036) Eq. 3-7; "Model Tells You What to
@@ -34,7 +35,8 @@
  *    every call leaves it zero-filled again, so one allocation serves many calls.
  *    Calls that share a workspace must be ordered on one stream.
  *  - Supported: head_dim d in {64, 128}; K/V/Q in bf16 or fp32
- *    (the same type for all three); decode needs G in {1, 2, 4}, scoring G*w <= 256;
+ *    (the same type for all three); decode needs G <= 8 (bf16) or G in {1, 2, 4}
+ *    (fp32); scoring needs G*w <= 256;
  *    all accumulation in fp32.
  */
 #ifndef KVC_H_
@@ -191,7 +193,8 @@ kvc_status kvc_append(const kvc_shape* shape, const void* k_new, const void* v_n
 /*
  * kvc_decode_attn - for query head h of slot s = h / G:
  *   out[h] = sum_{r < len[s]} softmax_r(q[h] . kp[off[s]+r] / sqrt(d)) vp[off[s]+r]
- *   (fp32 accumulation and output). Work is split evenly over the GPU by token
+ *   (fp32 accumulation and output; bf16 dot products on the tensor cores, fp32 on
+ *   the CUDA cores). Work is split evenly over the GPU by token
  *   ranges that may cross slot boundaries; partial results are merged by the last
  *   CTA to finish a slot. A slot with len 0 yields zeros.
  *   q [S*G, d] (dtype); kp, vp packed cache [kp_rows, d]; off [S+1]; len [S];
@@ -202,6 +205,20 @@ kvc_status kvc_decode_attn(const kvc_shape* shape, const void* q, const void* kp
                            const void* vp, const int64_t* off, const int32_t* len,
                            int64_t kp_rows, float* out, void* ws, size_t ws_bytes,
                            cudaStream_t stream);
+
+/*
+ * kvc_append_decode - kvc_append followed by kvc_decode_attn, fused into one launch
+ *   for bf16 (G <= 8): slot s with room gets its new token (k_new[s], v_new[s]) at
+ *   row off[s] + len[s], decode attends over len[s] + 1 rows including it, and len[s]
+ *   is incremented once every CTA has read it (by the last CTA to finish). A slot
+ *   without room (len == cap) is decoded over its old rows and flagged
+ *   KVC_DEVERR_APPEND_OVERFLOW, as with kvc_append. Other dtypes / G run the two calls.
+ *   Same workspace as kvc_decode_attn.
+ */
+kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const void* v_new,
+                             const void* q, void* kp, void* vp, const int64_t* off,
+                             const int32_t* cap, int32_t* len, int64_t kp_rows, float* out,
+                             void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /*
  * kvc_decode_attn_noalloc - kvc_decode_attn for callers that cannot allocate

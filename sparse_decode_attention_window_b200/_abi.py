@@ -21,7 +21,7 @@ KVC_WS_SCORE, KVC_WS_SELECT, KVC_WS_DECODE = 0, 1, 2
 # every symbol the header declares
 EXPORTS = ["kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout", "kvc_compact", "kvc_append",
            "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_last_error", "kvc_version",
-           "kvc_launch_count", "kvc_decode_attn_noalloc"]
+           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode"]
 
 
 class KvcShape(ctypes.Structure):
@@ -65,6 +65,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "kvc_version": (ctypes.c_char_p, []),
         "kvc_launch_count": (ctypes.c_ulonglong, []),
         "kvc_decode_attn_noalloc": (i32, [sh, vp, vp, vp, vp, vp, i64, vp, vp]),
+        "kvc_append_decode": (i32, [sh, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -30,39 +30,51 @@ __global__ void __launch_bounds__(1024) layout_kernel(const int32_t* __restrict_
 }
 
 // ---------------------------------------------------------------- compaction
-// Persistent grid over the packed rows; a group of TPR = row_bytes/16 threads
-// copies one row of K and one of V with 16-byte loads and stores. The slot of a
-// packed row is found by binary search over off[].
+// Persistent grid; CTA c owns the contiguous packed rows [c*R/grid, (c+1)*R/grid) of the
+// R = off[S] rows, so consecutive rows mostly share a slot: each row group finds the
+// slot of its first row by binary search once and then walks forward. A group of
+// TPR = row_bytes / 16 threads moves one K row and one V row with 16-byte accesses;
+// each group keeps UNROLL rows in flight.
 template <int TPR, int UNROLL>
-__global__ void __launch_bounds__(256) compact_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+__global__ void __launch_bounds__(256, 4) compact_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                       const int32_t* __restrict__ idx, int max_sel,
                                                       const int32_t* __restrict__ count,
                                                       const int64_t* __restrict__ off, int S, int L,
                                                       uint4* __restrict__ kp, uint4* __restrict__ vp,
                                                       int64_t kp_rows, int32_t* __restrict__ len) {
-  const long long gthreads = (long long)gridDim.x * blockDim.x;
   const long long gtid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (gtid < S) len[gtid] = min(max(count[gtid], 0), max_sel);
-  const int part = threadIdx.x % TPR;
-  const long long group = gtid / TPR, ngroups = gthreads / TPR;
+  constexpr int GROUPS = 256 / TPR;                 // row groups per CTA
+  const int part = threadIdx.x % TPR, grp = threadIdx.x / TPR;
   const long long total = off[S];
-  for (long long g0 = group; g0 < total; g0 += ngroups * UNROLL) {
+  const long long r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
+  if (r0 >= r1) return;
+  // slot of row r0: last s with off[s] <= r0
+  int s = 0;
+  {
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (off[mid] <= r0) lo = mid; else hi = mid - 1;
+    }
+    s = lo;
+  }
+  long long s_end = off[s + 1];
+  for (long long g0 = r0 + grp; g0 < r1; g0 += (long long)GROUPS * UNROLL) {
     uint4 kr[UNROLL], vr[UNROLL];
     long long dst[UNROLL];
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
       dst[u] = -1;
-      const long long g = g0 + (long long)u * ngroups;
-      if (g >= total) continue;
-      int lo = 0, hi = S - 1;            // last s with off[s] <= g
-      while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (off[mid] <= g) lo = mid; else hi = mid - 1;
+      const long long g = g0 + (long long)u * GROUPS;
+      if (g >= r1) continue;
+      while (g >= s_end && s < S - 1) {          // rows only increase: walk the slots forward
+        ++s;
+        s_end = off[s + 1];
       }
-      const int s = lo;
       const long long r = g - off[s];
       const int cnt = min(count[s], max_sel);
-      if (r >= cnt) continue;            // padding row: not written
+      if (r >= cnt) continue;                      // capacity padding: not written
       const int j = idx[(size_t)s * max_sel + r];
       if (j < 0 || j >= L || g >= kp_rows) {
         kvc_flag(KVC_DEVERR_INDEX_RANGE);

@@ -47,10 +47,10 @@ struct DecCfg {
 constexpr int DEC_MAX_SLOTS = 4096;
 
 template <typename T, int D, int G>
-constexpr size_t decode_smem_bytes(int S) {
+constexpr size_t decode_smem_bytes(int S, int grid) {
   using C = DecCfg<T, D, G>;
   return (size_t)C::STAGES * C::STAGE_BYTES + 2 * C::STAGES * sizeof(uint64_t) + (size_t)(S + 1) * sizeof(long long) +
-         (size_t)C::CONS_WARPS * (2 * G + G * D) * sizeof(float) + 16;
+         (size_t)C::CONS_WARPS * (2 * G + G * D) * sizeof(float) + (size_t)2 * grid * G * sizeof(float) + 16;
 }
 
 template <int G>
@@ -110,8 +110,64 @@ struct DecodeParams {
   float scale_log2;
   float* out;
   float* partial;   // [(gridDim.x + S) * G * (D + 2)]
-  int* counters;    // [S], zero on entry and on exit
+  int* counters;    // [S + 1], zero on entry and on exit ([S]: grid-wide ticket of the fused append)
+  // fused append (tensor-core kernel only): the new token of slot s is k_new[s], v_new[s]
+  int append;
+  const void* k_new;
+  const void* v_new;
+  const int32_t* cap;
+  int32_t* len_out;  // = len; incremented by the last CTA to finish
 };
+
+// The last CTA to finish slot s merges the slot's partials (CTAs cfirst..clast, stored
+// consecutively at index c + s) in one online pass: each thread owns output elements
+// e and folds the partials in groups of 8 whose (max, sum, value) loads are issued
+// together, so a merge of up to 8 partials costs one round trip to L2.
+KVC_DEV void merge_partials(const DecodeParams& a, int s, int G, int D, int cfirst, int clast, int tid, int nthr) {
+  const int np = clast - cfirst + 1;
+  const size_t stride = (size_t)G * (D + 2);
+  const float* base = a.partial + (size_t)(cfirst + s) * stride;
+  for (int e = tid; e < G * D; e += nthr) {
+    const int h = e / D;
+    float M = -INFINITY, Lt = 0.f, A = 0.f;
+    for (int i0 = 0; i0 < np; i0 += 8) {
+      float m[8], l[8], v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const bool in = i0 + k < np;
+        const float* pp = base + (size_t)(i0 + k) * stride;
+        m[k] = in ? __ldcg(pp + (size_t)G * D + h) : -INFINITY;
+        l[k] = in ? __ldcg(pp + (size_t)G * D + G + h) : 0.f;
+        v[k] = in ? __ldcg(pp + e) : 0.f;
+      }
+      float Mn = M;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) Mn = fmaxf(Mn, m[k]);
+      if (Mn == -INFINITY) continue;
+      const float sc = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      Lt *= sc;
+      A *= sc;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float w = m[k] == -INFINITY ? 0.f : exp2f(m[k] - Mn);
+        Lt += l[k] * w;
+        A += v[k] * w;
+      }
+      M = Mn;
+    }
+    a.out[(size_t)s * G * D + e] = Lt > 0.f ? A / Lt : 0.f;
+  }
+}
+
+// Ticket of slot s: returns true in the CTA that finishes the slot last. Called by one
+// thread after a CTA barrier that follows the CTA's partial writes; the acq_rel atomic
+// publishes them (release is cumulative over the barrier) and, in the last CTA, makes
+// the other CTAs' partials visible (acquire).
+KVC_DEV bool slot_ticket(int* counter, int last_value) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(counter), "r"(1) : "memory");
+  return old == last_value;
+}
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(DecCfg<T, D, G>::THREADS, 1) decode_kernel(DecodeParams a) {
@@ -369,31 +425,13 @@ __global__ void __launch_bounds__(DecCfg<T, D, G>::THREADS, 1) decode_kernel(Dec
       }
     }
     if (!single) {
-      __threadfence();
+      // the CTA's partial writes, then one fenced ticket (the barrier + one-thread fence
+      // orders every thread's writes before the atomic)
       named_bar_sync(1, C::CONS_WARPS * 32);
-      if (tid == 0) {
-        const int old = atomicAdd(&a.counters[s], 1);
-        last_flag = (old == clast - cfirst);
-      }
+      if (tid == 0) last_flag = slot_ticket(&a.counters[s], clast - cfirst);
       named_bar_sync(1, C::CONS_WARPS * 32);
       if (last_flag) {
-        __threadfence();
-        for (int e = tid; e < G * D; e += C::CONS_WARPS * 32) {
-          const int h = e / D;
-          float M = -INFINITY;
-          for (int cc = cfirst; cc <= clast; ++cc)
-            M = fmaxf(M, __ldcg(a.partial + (size_t)(cc + s) * G * (D + 2) + G * D + h));
-          float Lt = 0.f, A = 0.f;
-          for (int cc = cfirst; cc <= clast; ++cc) {
-            const float* pp = a.partial + (size_t)(cc + s) * G * (D + 2);
-            const float mw = __ldcg(pp + G * D + h);
-            if (mw == -INFINITY) continue;
-            const float sc = exp2f(mw - M);
-            Lt += __ldcg(pp + G * D + G + h) * sc;
-            A += __ldcg(pp + e) * sc;
-          }
-          a.out[(size_t)s * G * D + e] = Lt > 0.f ? A / Lt : 0.f;
-        }
+        merge_partials(a, s, G, D, cfirst, clast, tid, C::CONS_WARPS * 32);
         if (tid == 0) a.counters[s] = 0;
       }
     }

@@ -17,6 +17,7 @@
 #include "score_sm100.cuh"
 #include "select.cuh"
 #include "decode.cuh"
+#include "decode_mma.cuh"
 
 namespace {
 
@@ -113,6 +114,15 @@ bool force_simt() {
   return v;
 }
 
+// KVC_DECODE_PATH=simt routes bf16 decode to the CUDA-core kernel (cross-checks); read once.
+bool force_simt_decode() {
+  static const bool v = [] {
+    const char* e = getenv("KVC_DECODE_PATH");
+    return e && strcmp(e, "simt") == 0;
+  }();
+  return v;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -149,7 +159,7 @@ struct DecodeWs {
 DecodeWs decode_ws_layout(const kvc_shape* sh, int sms) {
   DecodeWs w{};
   w.cnt_off = 0;
-  w.cnt_bytes = align_up((size_t)sh->n_slots * sizeof(int), 256);
+  w.cnt_bytes = align_up((size_t)(sh->n_slots + 1) * sizeof(int), 256);
   w.part_off = w.cnt_bytes;
   w.part_bytes = align_up((size_t)(sms + sh->n_slots) * sh->G * (sh->d + 2) * sizeof(float), 256);
   w.total = w.part_off + w.part_bytes;
@@ -160,7 +170,7 @@ DecodeWs decode_ws_layout(const kvc_shape* sh, int sms) {
 template <typename T, int D, int G>
 kvc_status launch_decode(const kvc::DecodeParams& p, int sms, cudaStream_t st) {
   using namespace kvc;
-  const size_t smem = decode_smem_bytes<T, D, G>(p.S);
+  const size_t smem = decode_smem_bytes<T, D, G>(p.S, sms);
   DevInfo* di = nullptr;
   if (dev_info(&di) != KVC_OK) return KVC_ERR_CUDA;
   if (smem > (size_t)di->smem_optin)
@@ -173,6 +183,42 @@ kvc_status launch_decode(const kvc::DecodeParams& p, int sms, cudaStream_t st) {
   return check_launch("kvc_decode_attn");
 }
 
+// bf16: tensor-core decode (any G <= 8), K/V tiles by TMA through 2-D tensor maps of kp / vp
+template <int D>
+kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStream_t st) {
+  using namespace kvc;
+  DevInfo* di = nullptr;
+  if (dev_info(&di) != KVC_OK) return KVC_ERR_CUDA;
+  const size_t smem = decode_mma_smem_bytes<D>(p.S, G, sms);
+  if (smem > (size_t)di->smem_optin)
+    return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: %d slots need %zu B of shared memory (> %d)", p.S, smem,
+                di->smem_optin);
+  encode_tiled_fn enc = get_encode_tiled();
+  CUtensorMap mk64, mk16, mv64, mv16;
+  const long long rows = p.kp_rows > 0 ? p.kp_rows : 1;
+  if (!enc || !make_map_2d_rows(&mk64, enc, p.kp, D, rows, 64) || !make_map_2d_rows(&mk16, enc, p.kp, D, rows, 16) ||
+      !make_map_2d_rows(&mv64, enc, p.vp, D, rows, 64) || !make_map_2d_rows(&mv16, enc, p.vp, D, rows, 16))
+    return fail(KVC_ERR_CUDA, "kvc_decode_attn: cuTensorMapEncodeTiled failed");
+  kvc_status rc = set_smem(decode_mma_kernel<D>, smem, "kvc_decode_attn");
+  if (rc != KVC_OK) return rc;
+  // programmatic dependent launch: this grid may be scheduled while the previous kernel
+  // on the stream finishes; the kernel waits (griddepcontrol.wait) before reading inputs
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(DmCfg<D>::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mma_kernel<D>, mk64, mk16, mv64, mv16, p, G);
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "kvc_decode_attn: launch: %s", cudaGetErrorString(e));
+  count_launches(1);
+  return check_launch("kvc_decode_attn");
+}
+
 template <typename T, int D>
 kvc_status decode_by_g(int G, const kvc::DecodeParams& p, int sms, cudaStream_t st) {
   switch (G) {
@@ -181,6 +227,20 @@ kvc_status decode_by_g(int G, const kvc::DecodeParams& p, int sms, cudaStream_t 
     case 4: return launch_decode<T, D, 4>(p, sms, st);
     default: return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: G = %d (supported: 1, 2, 4)", G);
   }
+}
+
+// bf16 with G <= 8 -> tensor-core decode; otherwise the CUDA-core decode (G in {1, 2, 4}).
+kvc_status launch_decode_any(const kvc_shape* shape, const kvc::DecodeParams& p, int sms, cudaStream_t stream) {
+  if (shape->dtype == KVC_BF16 && shape->G <= 8 && !force_simt_decode()) {
+    if (shape->d == 128) return launch_decode_mma<128>(p, shape->G, sms, stream);
+    return launch_decode_mma<64>(p, shape->G, sms, stream);
+  }
+  if (shape->dtype == KVC_BF16) {
+    if (shape->d == 128) return decode_by_g<__nv_bfloat16, 128>(shape->G, p, sms, stream);
+    return decode_by_g<__nv_bfloat16, 64>(shape->G, p, sms, stream);
+  }
+  if (shape->d == 128) return decode_by_g<float, 128>(shape->G, p, sms, stream);
+  return decode_by_g<float, 64>(shape->G, p, sms, stream);
 }
 
 }  // namespace
@@ -457,12 +517,7 @@ kvc_status kvc_decode_attn(const kvc_shape* shape, const void* q, const void* kp
   p.out = out;
   p.partial = reinterpret_cast<float*>(wsb + w.part_off);
   p.counters = reinterpret_cast<int*>(wsb + w.cnt_off);
-  if (shape->dtype == KVC_BF16) {
-    if (shape->d == 128) return decode_by_g<__nv_bfloat16, 128>(shape->G, p, di->sms, stream);
-    return decode_by_g<__nv_bfloat16, 64>(shape->G, p, di->sms, stream);
-  }
-  if (shape->d == 128) return decode_by_g<float, 128>(shape->G, p, di->sms, stream);
-  return decode_by_g<float, 64>(shape->G, p, di->sms, stream);
+  return launch_decode_any(shape, p, di->sms, stream);
 }
 
 // Decode attention without a caller workspace: same kernel and results as
@@ -503,12 +558,49 @@ kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const 
   p.out = out;
   p.partial = reinterpret_cast<float*>(wsb + w.part_off);
   p.counters = reinterpret_cast<int*>(wsb + w.cnt_off);
-  if (shape->dtype == KVC_BF16) {
-    if (shape->d == 128) return decode_by_g<__nv_bfloat16, 128>(shape->G, p, di->sms, stream);
-    return decode_by_g<__nv_bfloat16, 64>(shape->G, p, di->sms, stream);
+  return launch_decode_any(shape, p, di->sms, stream);
+}
+
+kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const void* v_new, const void* q, void* kp,
+                             void* vp, const int64_t* off, const int32_t* cap, int32_t* len, int64_t kp_rows,
+                             float* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!k_new || !v_new || !q || !kp || !vp || !off || !cap || !len || !out)
+    return fail(KVC_ERR_INVALID_ARG, "kvc_append_decode: NULL pointer argument");
+  if (shape->dtype != KVC_BF16 || shape->G > 8 || force_simt_decode()) {
+    // the CUDA-core decode has no fused append: the two calls in sequence
+    if ((rc = kvc_append(shape, k_new, v_new, off, cap, len, kp, vp, kp_rows, stream)) != KVC_OK) return rc;
+    return kvc_decode_attn(shape, q, kp, vp, off, len, kp_rows, out, ws, ws_bytes, stream);
   }
-  if (shape->d == 128) return decode_by_g<float, 128>(shape->G, p, di->sms, stream);
-  return decode_by_g<float, 64>(shape->G, p, di->sms, stream);
+  if (shape->n_slots > kvc::DEC_MAX_SLOTS)
+    return fail(KVC_ERR_UNSUPPORTED, "kvc_append_decode: %d slots > %d", shape->n_slots, kvc::DEC_MAX_SLOTS);
+  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(ws) || !aligned16(k_new) || !aligned16(v_new))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_append_decode: buffers must be 16-byte aligned");
+  DevInfo* di = nullptr;
+  if ((rc = dev_info(&di)) != KVC_OK) return rc;
+  const DecodeWs w = decode_ws_layout(shape, di->sms);
+  if (!ws || ws_bytes < w.total)
+    return fail(KVC_ERR_WORKSPACE, "kvc_append_decode: workspace %zu B < required %zu B", ws_bytes, w.total);
+  unsigned char* wsb = static_cast<unsigned char*>(ws);
+  kvc::DecodeParams p{};
+  p.q = q;
+  p.kp = kp;
+  p.vp = vp;
+  p.off = off;
+  p.len = len;
+  p.kp_rows = kp_rows;
+  p.S = shape->n_slots;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)shape->d);
+  p.out = out;
+  p.partial = reinterpret_cast<float*>(wsb + w.part_off);
+  p.counters = reinterpret_cast<int*>(wsb + w.cnt_off);
+  p.append = 1;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.cap = cap;
+  p.len_out = len;
+  return launch_decode_any(shape, p, di->sms, stream);
 }
 
 }  // extern "C"

@@ -34,7 +34,8 @@ typedef kvc_status (*fail_fn)(kvc_status, const char*, ...);
 constexpr int TC_TILE = 128;      // keys per tile (MMA N in pass 1, M in pass 2)
 constexpr int TC_ROWS = 128;      // window rows per slot, padded (MMA M in pass 1, N in pass 2)
 constexpr int TC_STAGES = 4;
-constexpr int TC_THREADS = 192;   // 6 warps
+constexpr int TC_EPI_WARPS = 8;   // two per SM sub-partition; warp pair (w, w+4) splits the 128 columns
+constexpr int TC_THREADS = 32 * (2 + TC_EPI_WARPS);
 constexpr int TC_TMEM_COLS = 256; // two 128-column fp32 accumulators
 
 // ---------------------------------------------------------------- PTX wrappers (tcgen05)
@@ -82,6 +83,14 @@ KVC_DEV void tc_ld32(uint32_t taddr, float* v) {
 }
 KVC_DEV void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// 2^x on the special-function unit (approximate, subnormal results flushed to zero:
+// a probability below 2^-126 adds nothing to a softmax sum at fp32 precision).
+KVC_DEV float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Shared-memory matrix descriptor: K-major operand in the 128-byte swizzle layout
 // TMA writes (rows of 128 B, 8-row groups 1024 B apart), start 1024-B aligned.
 KVC_DEV uint64_t smem_desc_sw128(uint32_t saddr) {
@@ -116,7 +125,8 @@ struct TcSmem {
   static constexpr int NBAR = 2 * TC_STAGES + 2 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;     // tmem addr, flags
   static constexpr int LSE_OFF = MISC_OFF + 64;           // pass 2: lse2[128], win index [128]
-  static constexpr int TOTAL = LSE_OFF + 2 * TC_ROWS * 4;
+  static constexpr int XCH_OFF = LSE_OFF + 2 * TC_ROWS * 4; // half-to-half exchange [128] float2
+  static constexpr int TOTAL = XCH_OFF + TC_ROWS * 8;
   static constexpr int ALLOC = TOTAL + 1024;              // room to align the base to 1024 B
 };
 
@@ -165,9 +175,11 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L_::MISC_OFF + 4);
   float* lse_s = reinterpret_cast<float*>(sm + L_::LSE_OFF);
   int* win_s = reinterpret_cast<int*>(sm + L_::LSE_OFF + TC_ROWS * 4);
+  float2* xch = reinterpret_cast<float2*>(sm + L_::XCH_OFF);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.S * p.nsplit;
+  long long tiles_before = 0;   // epilogue: tiles of this CTA's earlier items
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < TC_STAGES; ++i) {
@@ -178,7 +190,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     mbar_init(q_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tm_full[b], 1);
-      mbar_init(&tm_empty[b], 4);
+      mbar_init(&tm_empty[b], TC_EPI_WARPS / 2);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -283,31 +295,42 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ epilogue: warps 2..5
-    const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    // ------------------------------------------------ epilogue: warps 2..9
+    // Two groups of four warps (one warp per SM sub-partition in each group) take the
+    // item's tiles in turn: group 0 the even tiles (TMEM accumulator 0), group 1 the odd
+    // ones (accumulator 1), so a thread always reads whole 128-column rows and no tile
+    // needs a cross-warp reduction. Warp w reads TMEM lanes 32*(w%4) .. +31.
+    const int ew = warp - 2;                      // 0..7
+    const int quarter = warp & 3;
+    const int grp = ew >> 2;                      // 0 or 1 = the TMEM accumulator this group reads
     const int t = quarter * 32 + lane;            // pass 1: window row; pass 2: key within the tile
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    int b = 0;
-    uint32_t tph = 0;
+    constexpr int NEPI = 32 * TC_EPI_WARPS;
+    uint32_t tph = 0;                             // phase of this group's accumulator barrier
     const int Lw = p.L - p.w;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const int s = item / p.nsplit, sp = item - s * p.nsplit;
       const int j0 = sp * p.tpi, j1 = min(p.tiles, j0 + p.tpi);
-      float m2 = -INFINITY, lsum = 0.f;            // pass 1 running stats of row t
+      float m2 = -INFINITY, lsum = 0.f;            // pass 1 running stats of row t over this group's tiles
       int vis = 0;
       if (PASS == 1) {
         vis = t < p.R ? visible_keys(p, Lw + (t % p.w)) : 0;
       } else {
-        named_bar_sync(1, 128);                     // previous item's lse_s reads are done
-        lse_s[t] = t < p.R ? p.lse2[(size_t)s * p.R + t] : INFINITY;
-        named_bar_sync(1, 128);
+        named_bar_sync(1, NEPI);                    // previous item's lse_s reads are done
+        if (grp == 0) lse_s[t] = t < p.R ? p.lse2[(size_t)s * p.R + t] : INFINITY;
+        named_bar_sync(1, NEPI);
       }
-      bool ok = true;
+      // the MMA warp alternates accumulators continuously across items: tile k of the
+      // CTA's sequence uses accumulator k & 1; this group takes the tiles with k & 1 == grp
       for (int j = j0; j < j1; ++j) {
-        if (!mbar_wait(&tm_full[b], tph) || *abort_flag) { ok = false; break; }
+        const long long k = tiles_before + (j - j0);
+        if ((int)(k & 1) != grp || !ok) continue;
+        if (!mbar_wait(&tm_full[grp], tph)) { ok = false; continue; }   // skip the rest, still meet below
+        tph ^= 1;
         tc_fence_after();
         float v[128];
-        const uint32_t ta = tmem_base + lane_base + (uint32_t)(b * 128);
+        const uint32_t ta = tmem_base + lane_base + (uint32_t)(grp * 128);
         tc_ld32(ta + 0, v);
         tc_ld32(ta + 32, v + 32);
         tc_ld32(ta + 64, v + 64);
@@ -315,32 +338,38 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tm_empty[b]);
-        if (++b == 2) { b = 0; tph ^= 1; }
+        if (lane == 0) mbar_arrive(&tm_empty[grp]);
 
         const int n0 = j * TC_TILE;
         if (PASS == 1) {
           if (t < p.R) {
-            const int nv = min(vis - n0, TC_TILE);    // visible columns of this tile
+            const int nv = min(vis - n0, TC_TILE);      // visible columns of this tile
             if (nv > 0) {
-              float mx = -INFINITY;
+              float mx[8];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) mx[c] = -INFINITY;
               if (nv == TC_TILE) {
 #pragma unroll
-                for (int c = 0; c < TC_TILE; ++c) mx = fmaxf(mx, v[c]);
+                for (int c = 0; c < TC_TILE; ++c) mx[c & 7] = fmaxf(mx[c & 7], v[c]);
               } else {
 #pragma unroll
-                for (int c = 0; c < TC_TILE; ++c) mx = c < nv ? fmaxf(mx, v[c]) : mx;
+                for (int c = 0; c < TC_TILE; ++c) mx[c & 7] = c < nv ? fmaxf(mx[c & 7], v[c]) : mx[c & 7];
               }
-              const float mnew = fmaxf(m2, mx * p.scale2);
-              float acc = 0.f;
+              const float mxa = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                      fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+              const float mnew = fmaxf(m2, mxa * p.scale2);
+              float acc[8];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) acc[c] = 0.f;
               if (nv == TC_TILE) {
 #pragma unroll
-                for (int c = 0; c < TC_TILE; ++c) acc += exp2f(fmaf(v[c], p.scale2, -mnew));
+                for (int c = 0; c < TC_TILE; ++c) acc[c & 7] += ex2_ftz(fmaf(v[c], p.scale2, -mnew));
               } else {
 #pragma unroll
-                for (int c = 0; c < TC_TILE; ++c) acc += c < nv ? exp2f(fmaf(v[c], p.scale2, -mnew)) : 0.f;
+                for (int c = 0; c < TC_TILE; ++c) acc[c & 7] += c < nv ? ex2_ftz(fmaf(v[c], p.scale2, -mnew)) : 0.f;
               }
-              lsum = lsum * exp2f(m2 - mnew) + acc;
+              const float at = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+              lsum = lsum * ex2_ftz(m2 - mnew) + at;
               m2 = mnew;
             }
           }
@@ -349,27 +378,44 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
           if (n < p.N) {
             const int pos = p.key_pos ? p.key_pos[n] : n;
             const int imin = pos - Lw;                 // rows with window index >= imin see the key
-            float acc = 0.f;
+            float acc[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) acc[c] = 0.f;
             if (imin <= 0) {
 #pragma unroll
               for (int c = 0; c < TC_ROWS; c += 4) {
                 const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c);
-                acc += exp2f(fmaf(v[c + 0], p.scale2, -l4.x));
-                acc += exp2f(fmaf(v[c + 1], p.scale2, -l4.y));
-                acc += exp2f(fmaf(v[c + 2], p.scale2, -l4.z));
-                acc += exp2f(fmaf(v[c + 3], p.scale2, -l4.w));
+                acc[(c + 0) & 7] += ex2_ftz(fmaf(v[c + 0], p.scale2, -l4.x));
+                acc[(c + 1) & 7] += ex2_ftz(fmaf(v[c + 1], p.scale2, -l4.y));
+                acc[(c + 2) & 7] += ex2_ftz(fmaf(v[c + 2], p.scale2, -l4.z));
+                acc[(c + 3) & 7] += ex2_ftz(fmaf(v[c + 3], p.scale2, -l4.w));
               }
             } else {
 #pragma unroll
               for (int c = 0; c < TC_ROWS; ++c)
-                acc += win_s[c] >= imin ? exp2f(fmaf(v[c], p.scale2, -lse_s[c])) : 0.f;
+                acc[c & 7] += win_s[c] >= imin ? ex2_ftz(fmaf(v[c], p.scale2, -lse_s[c])) : 0.f;
             }
-            p.score[(size_t)s * p.N + n] = acc;
+            p.score[(size_t)s * p.N + n] =
+                ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
           }
         }
       }
-      if (!ok) break;
-      if (PASS == 1 && t < p.R) p.part[((size_t)s * p.nsplit + sp) * p.R + t] = make_float2(m2, lsum);
+      tiles_before += j1 - j0;
+      // both groups meet here whatever happened; any failed wait stops every epilogue warp
+      if (named_bar_or(2, NEPI, !ok)) { ok = false; break; }
+      if (PASS == 1) {
+        // merge the two groups' running stats of row t, then write the item's partial
+        if (grp == 1) xch[t] = make_float2(m2, lsum);
+        named_bar_sync(2, NEPI);
+        if (grp == 0 && t < p.R) {
+          const float2 o = xch[t];
+          const float M = fmaxf(m2, o.x);
+          float l = 0.f;
+          if (M != -INFINITY)
+            l = (m2 == -INFINITY ? 0.f : lsum * ex2_ftz(m2 - M)) + (o.x == -INFINITY ? 0.f : o.y * ex2_ftz(o.x - M));
+          p.part[((size_t)s * p.nsplit + sp) * p.R + t] = make_float2(M, l);
+        }
+      }
     }
   }
 

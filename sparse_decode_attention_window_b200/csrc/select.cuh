@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
   const float* sc = a.score + (size_t)s * N;
   const int32_t* ce = a.chunk_end;
   const bool cached = N <= a.key_cap;
+  const bool unit = !chunk && !massc;      // top-B: unit weights
   if (!a.score || (chunk && !ce) || (!massc && !idx_row) || (pol != KVC_POL_TOPB && !massc && !chunk)) {
     // a policy whose inputs are missing (or an unknown policy code): keep nothing, report it
     if (tid == 0) { kvc_flag(KVC_DEVERR_INDEX_RANGE); a.count[s] = 0; }
@@ -209,20 +210,25 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
       if (match) {
         const unsigned peers = __match_any_sync(mm, bin);
         const int leader = __ffs(peers) - 1;
-        sh.wstage[tid] = wt;
-        __syncwarp(mm);
-        if (lane == leader) {
-          unsigned long long sum = 0;
-          unsigned rest = peers;
-          while (rest) {
-            int l = __ffs(rest) - 1;
-            rest &= rest - 1;
-            sum += sh.wstage[(tid & ~31) + l];
+        if (unit) {
+          // top-B: every weight is 1, the count is the weight
+          if (lane == leader) atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
+        } else {
+          sh.wstage[tid] = wt;
+          __syncwarp(mm);
+          if (lane == leader) {
+            unsigned long long sum = 0;
+            unsigned rest = peers;
+            while (rest) {
+              int l = __ffs(rest) - 1;
+              rest &= rest - 1;
+              sum += sh.wstage[(tid & ~31) + l];
+            }
+            atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
+            atomicAdd(&sh.hw[bin], sum);
           }
-          atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
-          atomicAdd(&sh.hw[bin], sum);
+          __syncwarp(mm);
         }
-        __syncwarp(mm);
       }
     }
     __syncthreads();
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     const int lo = max(hi - per, 0);
     unsigned long long my_w = 0;
     uint32_t my_c = 0;
-    for (int b = hi - 1; b >= lo; --b) { my_w += sh.hw[b]; my_c += sh.hcnt[b]; }
+    for (int b = hi - 1; b >= lo; --b) { my_w += unit ? sh.hcnt[b] : sh.hw[b]; my_c += sh.hcnt[b]; }
     unsigned long long tot_w;
     uint32_t tot_c;
     unsigned long long before_w = block_exclusive_scan<unsigned long long>(hi > lo ? my_w : 0ull, sh.scan64, &tot_w);
@@ -241,8 +247,8 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
       unsigned long long run = w_above + before_w;
       uint32_t runc = before_c;
       for (int b = hi - 1; b >= lo; --b) {
-        const unsigned long long wb = sh.hw[b];
         const uint32_t cb = sh.hcnt[b];
+        const unsigned long long wb = unit ? (unsigned long long)cb : sh.hw[b];
         if (cb > 0 && run < target && run + wb >= target) {
           sh.sel_bin = b;
           sh.w_above_bin = run;

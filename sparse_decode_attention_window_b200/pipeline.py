@@ -9,6 +9,7 @@ from __future__ import annotations
 import torch
 
 from . import (kvc_score, kvc_select, kvc_alloc_budgets, kvc_layout, kvc_compact, kvc_append, kvc_decode_attn,
+               kvc_append_decode,
                kvc_workspace_size, make_shape, KVC_WS_SCORE, KVC_WS_DECODE, KVC_POL_TOPB, KVC_POL_MASS_COUNT,
                KVC_POL_CHUNK)
 
@@ -105,14 +106,20 @@ class KvcPipeline:
         self.select_step(stream)
         self.compact_step(stream)
 
-    def decode_step(self, t: int, q=None, k_new=None, v_new=None, out=None, stream=None):
+    def decode_step(self, t: int, q=None, k_new=None, v_new=None, out=None, fused=True, stream=None):
+        """Append the step's new token to every slot, then decode. `fused` uses the
+        one-launch kvc_append_decode; otherwise kvc_append then kvc_decode_attn."""
         inp = self.inp
         q = inp.q_dec[t] if q is None else q
         k_new = inp.k_dec[t] if k_new is None else k_new
         v_new = inp.v_dec[t] if v_new is None else v_new
         out = self.out if out is None else out
-        kvc_append(self.shape, k_new, v_new, self.off, self.cap, self.len, self.kp, self.vp, stream=stream)
-        kvc_decode_attn(self.shape, q, self.kp, self.vp, self.off, self.len, out, self.ws_decode, stream=stream)
+        if fused:
+            kvc_append_decode(self.shape, k_new, v_new, q, self.kp, self.vp, self.off, self.cap, self.len, out,
+                              self.ws_decode, stream=stream)
+        else:
+            kvc_append(self.shape, k_new, v_new, self.off, self.cap, self.len, self.kp, self.vp, stream=stream)
+            kvc_decode_attn(self.shape, q, self.kp, self.vp, self.off, self.len, out, self.ws_decode, stream=stream)
         return out
 
     def run(self, steps=None, record=False, stream=None):

@@ -26,7 +26,7 @@ def _np(t):
     return t.detach().cpu().numpy()
 
 
-def run_and_check(wl, slots=None, steps=None, gen_device="cpu", check_scores=True):
+def run_and_check(wl, slots=None, steps=None, gen_device="cpu", check_scores=True, fused=True):
     """Run the workload through the ABI and check it against the oracle.
     slots: slots to check (default all); steps: decode steps to check (default all)."""
     from sparse_decode_attention_window_b200.pipeline import KvcPipeline
@@ -111,7 +111,7 @@ def run_and_check(wl, slots=None, steps=None, gen_device="cpu", check_scores=Tru
     want_steps = set(steps)
     outs = {}
     for t in range(max(steps) + 1 if steps else 0):
-        o_t = pipe.decode_step(t)
+        o_t = pipe.decode_step(t, fused=fused)
         if t in want_steps:
             outs[t] = _np(o_t).copy()
     torch.cuda.synchronize()
@@ -298,17 +298,64 @@ def test_decode_is_independent_of_how_tokens_split_over_ctas():
 
 
 def test_wide_window_takes_cuda_core_scoring_path():
-    """G*w = 256 rows exceeds the tensor-core tile: scoring runs on the CUDA-core kernels."""
-    run_and_check(get("llama8b").scaled(batch=1, hq=16, hkv=2, L=900, w=32, top_b=100, steps=0), steps=[])
+    """G*w = 256 rows exceeds the tensor-core tile: scoring runs on the CUDA-core kernels;
+    decode with G = 8 query heads per KV head."""
+    run_and_check(get("llama8b").scaled(batch=1, hq=16, hkv=2, L=900, w=32, top_b=100, steps=3))
 
 
-def test_cuda_core_scoring_path_on_bf16_workloads():
-    """The CUDA-core scoring kernels, forced for bf16, pass the same oracle checks."""
+def test_cuda_core_paths_on_bf16_workloads():
+    """The CUDA-core scoring and decode kernels, forced for bf16, pass the same oracle checks."""
     import os
     import subprocess
     import sys
-    env = dict(os.environ, KVC_SCORE_PATH="simt")
+    env = dict(os.environ, KVC_SCORE_PATH="simt", KVC_DECODE_PATH="simt")
     r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
-                        "-k", "llama8b_shape_small_context or zigzag_small or chunk_small"],
+                        "-k", "llama8b_shape_small_context or zigzag_small or chunk_small or fastgen_small "
+                              "or decode_is_independent"],
                        env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+@pytest.mark.parametrize("name,kw", [("llama8b", dict(batch=2, L=1500, top_b=200, steps=4)),
+                                     ("fastgen", dict(batch=2, L=2000, steps=4)),
+                                     ("tiny", dict())])
+def test_separate_append_then_decode_calls(name, kw):
+    """kvc_append followed by kvc_decode_attn (two launches) gives the same results."""
+    run_and_check(get(name).scaled(**kw), fused=False)
+
+
+def test_fused_append_decode_overflow_keeps_old_rows():
+    import sparse_decode_attention_window_b200 as kvc
+    S, G, d = 3, 4, 128
+    sh = kvc.make_shape(S, G, d, 64, 0, S, 1, torch.bfloat16)
+    count = torch.tensor([16, 5, 0], dtype=torch.int32, device="cuda")
+    off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    cap = torch.empty(S, dtype=torch.int32, device="cuda")
+    kvc.kvc_layout(count, 0, off, cap)          # caps 16, 16, 0: slot 0 full, slot 2 has no room
+    rows = int(off[-1])
+    kp = torch.randn(rows, d, device="cuda").to(torch.bfloat16)
+    vp = torch.randn(rows, d, device="cuda").to(torch.bfloat16)
+    kp0, vp0 = kp.clone(), vp.clone()
+    ln = count.clone()
+    q = torch.randn(S * G, d, device="cuda").to(torch.bfloat16)
+    kn = torch.randn(S, d, device="cuda").to(torch.bfloat16)
+    vn = torch.randn(S, d, device="cuda").to(torch.bfloat16)
+    out = torch.empty((S * G, d), device="cuda")
+    ws = torch.zeros(kvc.kvc_workspace_size(kvc.KVC_WS_DECODE, sh), dtype=torch.uint8, device="cuda")
+    kvc.kvc_append_decode(sh, kn, vn, q, kp, vp, off, cap, ln, out, ws)
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.kvc_get_status()
+    assert "append-overflow" in str(e.value)
+    assert ln.cpu().tolist() == [16, 6, 0]
+    # slot 1 got its token at row off[1] + 5; slot 0's rows are untouched
+    assert torch.equal(kp[16 + 5], kn[1]) and torch.equal(vp[16 + 5], vn[1])
+    assert torch.equal(kp[:16], kp0[:16])
+    o = _np(out)
+    ref0 = O.decode_attention(q[0:G].cpu(), kp0[:16].cpu(), vp0[:16].cpu(), [0, 16], [16], G)
+    keys1 = torch.cat([kp0[16:21], kn[1:2]]).cpu()
+    vals1 = torch.cat([vp0[16:21], vn[1:2]]).cpu()
+    ref1 = O.decode_attention(q[G:2 * G].cpu(), keys1, vals1, [0, 6], [6], G)
+    P.check_out(o[0:G], ref0, "bf16", "full slot")
+    P.check_out(o[G:2 * G], ref1, "bf16", "appended slot")
+    assert (o[2 * G:] == 0).all()
+    kvc.kvc_get_status()
