@@ -274,3 +274,69 @@ def decode_attention(q, kp, vp, off, length, G: int) -> np.ndarray:
         p /= p.sum()
         out[h] = p @ vs
     return out
+
+
+# ---------------------------------------------------------------------------
+# next rows: attention loss (ZigZagKV Section 5.5, Table 3) and head profiling
+# ---------------------------------------------------------------------------
+def retained_mass(score, kept) -> float:
+    """Share of a head's window-attention mass that the kept tokens hold:
+    sum_{j in kept} score_j / sum_j score_j (0 for a head with no mass)."""
+    sc = _f64(score)
+    total = sc.sum()
+    if total <= 0:
+        return 0.0
+    return float(sc[np.asarray(kept, dtype=np.int64)].sum() / total)
+
+
+def attention_loss(retained, target: float = 0.9) -> float:
+    """ZigZagKV's attention loss of one head: how far the retained mass falls short of
+    the 0.9 the LMBA budget is defined by (0 when it reaches it). Reading: the page
+    calls it the average deviation from achieving 0.9 attention; a head above 0.9
+    deviates by nothing."""
+    return max(0.0, float(target) - float(retained))
+
+
+def profile_head(score, special_mask_row, window: int, tau: float) -> int:
+    """FastGen-style head profiling from window attention (the pages give no
+    criterion; this is the reading): among the policies local (keep the last
+    `window` tokens), special (keep the special tokens) and full, pick the one that
+    keeps the fewest tokens while retaining at least `tau` of the head's attention
+    mass; ties in size go local, then special. Returns the policy code."""
+    sc = _f64(score)
+    L = sc.shape[0]
+    cands = []
+    loc = local_indices(L, window)
+    cands.append((len(loc), 0, 2, loc))                  # LOCAL
+    spc = special_indices(special_mask_row)
+    cands.append((len(spc), 1, 3, spc))                  # SPECIAL
+    for size, order, code, idx in sorted(cands, key=lambda c: (c[0], c[1])):
+        if retained_mass(sc, idx) >= tau:
+            return code
+    return 4                                             # FULL
+
+
+def chunk_select_local(cscore, chunk_end, target_tokens: int, n_local: int):
+    """ChunkLLM chunk selection with always-kept local chunks (its Section 3.2 keeps
+    the 15 or 16 most recent chunks): the last n_local chunks are kept, then the
+    other chunks in score order (descending, ties by chunk index) until the kept
+    chunks hold at least `target_tokens` tokens. Returns (tokens ascending, chunk ids ascending)."""
+    sc = _f64(cscore)
+    ends = np.asarray(chunk_end, dtype=np.int64)
+    C = ends.shape[0]
+    starts = np.concatenate([[0], ends[:-1] + 1])
+    lens = ends - starts + 1
+    n_local = max(0, min(int(n_local), C))
+    forced = np.arange(C - n_local, C, dtype=np.int64)
+    have = int(lens[forced].sum())
+    rest = np.arange(0, C - n_local, dtype=np.int64)
+    chosen = list(forced)
+    if have < target_tokens and rest.size:
+        order = rest[_desc_order(sc[rest])]
+        cum = have + np.cumsum(lens[order])
+        n = min(int(np.searchsorted(cum, int(target_tokens), side="left")) + 1, order.size)
+        chosen += list(order[:n])
+    chosen = np.sort(np.asarray(chosen, dtype=np.int64))
+    toks = (np.concatenate([np.arange(starts[c], ends[c] + 1) for c in chosen]).astype(np.int64)
+            if chosen.size else np.zeros(0, dtype=np.int64))
+    return toks, chosen

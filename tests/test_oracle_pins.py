@@ -333,3 +333,76 @@ def test_tiny_workload_sinks_are_kept():
     res = run_workload(make_inputs(wl, "cpu"), steps=0)
     for s in range(wl.n_slots):
         assert {0, 1, 2, 3} <= set(res.sel[s].tolist())
+
+
+# ---------------------------------------------------------------- next rows
+def test_retained_mass_limits_and_lmba_consistency():
+    r = _rng(300)
+    sc = r.random(200) ** 4
+    assert O.retained_mass(sc, np.arange(200)) == pytest.approx(1.0, abs=1e-15)
+    assert O.retained_mass(sc, np.array([], dtype=np.int64)) == 0.0
+    assert O.retained_mass(np.zeros(5), [0, 1]) == 0.0
+    # the LMBA count is exactly where the top-k retained mass first reaches 0.9
+    k = O.mass_count(sc, 0.9)
+    assert O.retained_mass(sc, O.top_b(sc, k)) >= 0.9
+    assert O.retained_mass(sc, O.top_b(sc, k - 1)) < 0.9
+    assert O.attention_loss(O.retained_mass(sc, O.top_b(sc, k))) == 0.0
+    assert O.attention_loss(0.5) == pytest.approx(0.4)
+
+
+def test_top_b_retains_the_most_mass_brute_force():
+    r = _rng(301)
+    for _ in range(10):
+        n = int(r.integers(3, 11))
+        sc = r.random(n)
+        for B in range(1, n + 1):
+            best = max(O.retained_mass(sc, list(c)) for c in itertools.combinations(range(n), B))
+            assert O.retained_mass(sc, O.top_b(sc, B)) == pytest.approx(best, rel=1e-12)
+
+
+def test_profile_head_picks_the_cheapest_sufficient_policy():
+    L, W = 100, 10
+    mask = np.zeros(L, np.uint8); mask[[0, 1, 2, 3, 50]] = 1           # 5 special tokens
+    local = np.zeros(L); local[90:] = 1.0                               # all mass in the window
+    assert O.profile_head(local, mask, W, 0.95) == 2                    # LOCAL
+    special = np.zeros(L); special[[0, 1, 2, 3, 50]] = 1.0
+    assert O.profile_head(special, mask, W, 0.95) == 3                  # SPECIAL (5 tokens, cheaper than 10)
+    both = np.zeros(L); both[[0, 1, 2, 3, 50]] = 1.0; both[95] = 1000.0   # most mass in the window
+    assert O.profile_head(both, mask, W, 0.95) == 2
+    flat = np.ones(L)
+    assert O.profile_head(flat, mask, W, 0.95) == 4                     # FULL
+    # with fewer special tokens than the window, special is tried first
+    assert O.profile_head(special + local * 1e-9, mask, W, 0.95) == 3
+
+
+def test_chunk_select_local_reduces_and_forces():
+    r = _rng(302)
+    for _ in range(30):
+        L = int(r.integers(5, 80))
+        cuts = np.sort(r.choice(np.arange(L - 1), size=int(r.integers(0, L - 1)), replace=False))
+        ends = np.concatenate([cuts, [L - 1]])
+        C = len(ends)
+        sc = r.random(C)
+        target = int(r.integers(1, L + 1))
+        # no local chunks: the plain selection
+        t0, c0 = O.chunk_select_local(sc, ends, target, 0)
+        t1, c1 = O.chunk_select(sc, ends, target)
+        np.testing.assert_array_equal(t0, t1)
+        nl = int(r.integers(0, C + 1))
+        toks, chosen = O.chunk_select_local(sc, ends, target, nl)
+        lens = np.diff(np.concatenate([[-1], ends]))
+        assert set(range(C - nl, C)) <= set(chosen.tolist())          # local chunks always kept
+        assert len(toks) == lens[chosen].sum()
+        assert len(toks) >= min(target, L) or len(chosen) == C
+        free = [c for c in chosen if c < C - nl]
+        if free:                                                         # minimal: the worst free chunk was needed
+            worst = free[int(np.argmin(sc[free]))]
+            assert lens[chosen].sum() - lens[worst] < target
+            # the free chunks are the top chunks by score among the non-local ones
+            others = np.arange(C - nl)
+            top = np.sort(others[np.argsort(-sc[others], kind="stable")[: len(free)]])
+            np.testing.assert_array_equal(np.sort(free), top)
+    # every chunk local: everything kept
+    ends = np.array([2, 5, 9])
+    toks, chosen = O.chunk_select_local(np.array([0.1, 0.2, 0.3]), ends, 1, 3)
+    np.testing.assert_array_equal(toks, np.arange(10))
