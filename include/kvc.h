@@ -240,6 +240,42 @@ kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const 
                                    const void* vp, const int64_t* off, const int32_t* len,
                                    int64_t kp_rows, float* out, cudaStream_t stream);
 
+/*
+ * kvc_select_chunks - ChunkLLM chunk selection with always-kept local chunks (ChunkLLM
+ *   Section 3.2 keeps the 15 or 16 most recent chunks): for every slot, the last
+ *   n_local chunks are kept, then the other chunks in descending chunk-score order
+ *   (ties: lower chunk index) until the kept chunks hold >= target[s] tokens; every
+ *   token of the kept chunks is written to idx[s] in ascending order. With n_local = 0
+ *   this is kvc_select's KVC_POL_CHUNK.
+ *   chunk_score [S, C] fp32; chunk_end [C]; target [S] int32; idx [S, max_sel]; count [S].
+ */
+kvc_status kvc_select_chunks(const kvc_shape* shape, const float* chunk_score, const int32_t* chunk_end,
+                             int32_t C, const int32_t* target, int32_t n_local, int32_t* idx,
+                             int32_t max_sel, int32_t* count, cudaStream_t stream);
+
+/*
+ * kvc_retained_mass - share of each slot's window-attention mass its kept tokens hold:
+ *   retained[s] = sum_{r < count[s]} score[s][idx[s][r]] / sum_n score[s][n] (0 if no
+ *   mass). ZigZagKV's attention loss (Section 5.5, Table 3) is max(0, 0.9 - retained).
+ *   score [S, N] fp32; idx [S, max_sel]; count [S]; retained [S] fp32 out (fp64 sums).
+ */
+kvc_status kvc_retained_mass(const kvc_shape* shape, const float* score, int32_t N, const int32_t* idx,
+                             int32_t max_sel, const int32_t* count, float* retained, cudaStream_t stream);
+
+/*
+ * kvc_profile_heads - FastGen-style head profiling from the window scores (FastGen
+ *   abstract / Section 1: profile the heads, then give local heads a recent window,
+ *   special-token heads the special tokens, broad heads the full cache). The pages
+ *   give no criterion; this one keeps the policy (local: the last `window` tokens;
+ *   special: the batch row's special tokens) that keeps fewer tokens (ties: local)
+ *   among those whose share of the head's window-attention mass is >= tau, else full.
+ *   policy [S] int8 out (feeds kvc_select); shares [S][2] fp32 out or NULL: the local
+ *   and special mass shares. special_mask [batch, L] or NULL (no special policy).
+ */
+kvc_status kvc_profile_heads(const kvc_shape* shape, const float* score, const uint8_t* special_mask,
+                             int32_t window, float tau, int8_t* policy, float* shares,
+                             cudaStream_t stream);
+
 /* Bytes of workspace the call `which` (KVC_WS_*) needs for this shape (C: chunks, 0 if none). */
 size_t kvc_workspace_size(int which, const kvc_shape* shape, int32_t C);
 

@@ -18,7 +18,8 @@ from ._abi import (KvcShape, KvcError, KVC_BF16, KVC_FP32, KVC_POL_TOPB, KVC_POL
 
 __all__ = ["KvcShape", "KvcError", "make_shape", "kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout",
            "kvc_compact", "kvc_append", "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_version",
-           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode",
+           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_select_chunks",
+           "kvc_retained_mass", "kvc_profile_heads",
            "library", "KVC_BF16", "KVC_FP32", "KVC_POL_TOPB", "KVC_POL_MASS_COUNT", "KVC_POL_LOCAL",
            "KVC_POL_SPECIAL", "KVC_POL_FULL", "KVC_POL_CHUNK", "KVC_WS_SCORE", "KVC_WS_SELECT", "KVC_WS_DECODE"]
 
@@ -111,6 +112,25 @@ def kvc_decode_attn_noalloc(shape, q, kp, vp, off, length, out, stream=None):
     _check("kvc_decode_attn_noalloc",
            library().kvc_decode_attn_noalloc(ctypes.byref(shape), _ptr(q), _ptr(kp), _ptr(vp), _ptr(off),
                                              _ptr(length), int(kp.shape[0]), _ptr(out), _stream(stream)))
+
+
+def kvc_select_chunks(shape, chunk_score, chunk_end, target, idx, count, n_local=0, stream=None):
+    _check("kvc_select_chunks",
+           library().kvc_select_chunks(ctypes.byref(shape), _ptr(chunk_score), _ptr(chunk_end),
+                                       int(chunk_end.numel()), _ptr(target), int(n_local), _ptr(idx),
+                                       int(idx.shape[-1]), _ptr(count), _stream(stream)))
+
+
+def kvc_retained_mass(shape, score, idx, count, retained, stream=None):
+    _check("kvc_retained_mass",
+           library().kvc_retained_mass(ctypes.byref(shape), _ptr(score), int(score.shape[-1]), _ptr(idx),
+                                       int(idx.shape[-1]), _ptr(count), _ptr(retained), _stream(stream)))
+
+
+def kvc_profile_heads(shape, score, policy, window, tau=0.95, special_mask=None, shares=None, stream=None):
+    _check("kvc_profile_heads",
+           library().kvc_profile_heads(ctypes.byref(shape), _ptr(score), _ptr(special_mask), int(window),
+                                       float(tau), _ptr(policy), _ptr(shares), _stream(stream)))
 
 
 def kvc_get_status(stream=None):

@@ -21,7 +21,8 @@ KVC_WS_SCORE, KVC_WS_SELECT, KVC_WS_DECODE = 0, 1, 2
 # every symbol the header declares
 EXPORTS = ["kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout", "kvc_compact", "kvc_append",
            "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_last_error", "kvc_version",
-           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode"]
+           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_select_chunks",
+           "kvc_retained_mass", "kvc_profile_heads"]
 
 
 class KvcShape(ctypes.Structure):
@@ -66,6 +67,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "kvc_launch_count": (ctypes.c_ulonglong, []),
         "kvc_decode_attn_noalloc": (i32, [sh, vp, vp, vp, vp, vp, i64, vp, vp]),
         "kvc_append_decode": (i32, [sh, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
+        "kvc_select_chunks": (i32, [sh, vp, vp, i32, vp, i32, vp, i32, vp, vp]),
+        "kvc_retained_mass": (i32, [sh, vp, i32, vp, i32, vp, vp, vp]),
+        "kvc_profile_heads": (i32, [sh, vp, vp, i32, f32, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -15,7 +15,8 @@ LIB = os.path.join(HERE, "libkvc.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 SOURCES = ["kvc.cu"]
-HEADERS = ["common.cuh", "score_simt.cuh", "score_sm100.cuh", "select.cuh", "cache.cuh", "decode.cuh"]
+# every header under csrc/ (the unity build includes them all)
+HEADERS = sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))
 
 
 def nvcc_path() -> str:

@@ -44,7 +44,7 @@ constexpr size_t decode_mma_smem_bytes(int S, int G, int grid) {
   using C = DmCfg<D>;
   return 1024 + (size_t)C::STAGES * C::STAGE_BYTES + 2 * C::STAGES * sizeof(uint64_t) +
          (size_t)(2 * S + 1) * sizeof(long long) + (size_t)C::CONS_WARPS * (2 * G + G * D) * sizeof(float) +
-         (size_t)2 * grid * G * sizeof(float) + (size_t)S + 16;
+         (size_t)2 * grid * G * sizeof(float) + (size_t)G * (D + 2) * sizeof(float) + (size_t)S + 16;
 }
 
 KVC_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -76,6 +76,23 @@ KVC_DEV uint32_t pack_bf16(float lo, float hi) {
 }
 KVC_DEV float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
+KVC_DEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+KVC_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Read a float from the same shared-memory offset in CTA `rank` of this cluster.
+KVC_DEV float ld_dsmem(const float* local, uint32_t rank) {
+  uint32_t ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
 // Byte offset of (row, 16-byte chunk) in a 128-byte-swizzled region of 128-byte rows.
 KVC_DEV uint32_t swz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
 
@@ -99,11 +116,19 @@ KVC_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
       : "memory");
 }
 
+// Two ways to split the work, chosen on the device from the lengths (every CTA reads
+// all of them and reaches the same choice):
+//  * per-slot clusters - when the grid was launched in clusters of k CTAs, every slot
+//    fits one cluster, the clusters cover >= 3/4 of the grid and the lengths are near
+//    uniform (max * S <= 1.25 * total): slot j gets cluster j, whose k CTAs split its
+//    tokens evenly and merge their k partials through distributed shared memory;
+//  * token ranges - otherwise: the valid tokens of all slots are cut into gridDim.x
+//    equal ranges (ranges may cross slots) and partials merge through global tickets.
 template <int D>
 __global__ void __launch_bounds__(DmCfg<D>::THREADS, 1)
 decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constant__ CUtensorMap mk16,
                   const __grid_constant__ CUtensorMap mv64, const __grid_constant__ CUtensorMap mv16,
-                  DecodeParams a, int G) {
+                  DecodeParams a, int G, int ksz) {
   using C = DmCfg<D>;
   extern __shared__ __align__(1024) unsigned char dm_raw[];
   const uint32_t raw = smem_u32(dm_raw);
@@ -114,12 +139,16 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   long long* P = reinterpret_cast<long long*>(empty + C::STAGES);
   long long* offs = P + a.S + 1;                          // off[] of the slots
   float* comb = reinterpret_cast<float*>(offs + a.S);    // [warps][2G + G*D]
-  unsigned char* app = reinterpret_cast<unsigned char*>(comb + C::CONS_WARPS * (2 * G + G * D) + 2 * gridDim.x * G);
+  float* cres = comb + C::CONS_WARPS * (2 * G + G * D) + 2 * gridDim.x * G;   // cluster mode: acc[G*D], m[G], l[G]
+  unsigned char* app = reinterpret_cast<unsigned char*>(cres + G * (D + 2));
   __shared__ unsigned long long scan_sh[33];
   __shared__ int last_flag;
   __shared__ int abort_flag;
+  __shared__ unsigned long long max_len_sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) max_len_sh = 0;
+  __syncthreads();
   const int S = a.S;
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
 
@@ -129,33 +158,46 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // prefix of the valid lengths over slots (lengths clipped to the buffer); with the
-  // fused append, a slot that has room gets its new token as its last row
-  unsigned long long carry = 0;
+  // One slot's length (clipped to the buffer); with the fused append, a slot that has
+  // room gets its new token as its last row.
+  auto slot_len = [&](int s, unsigned char* ap_out, bool flag_overflow) -> long long {
+    long long n = max(a.len[s], 0);
+    const long long os = a.off[s];
+    offs[s] = os;
+    const long long room = a.kp_rows - os;
+    if (n > room) { kvc_flag(KVC_DEVERR_INDEX_RANGE); n = room > 0 ? room : 0; }
+    unsigned char ap = 0;
+    if (a.append) {
+      if (a.len[s] >= 0 && n < a.cap[s] && n < room) { ap = 1; ++n; }
+      else if (flag_overflow) kvc_flag(KVC_DEVERR_APPEND_OVERFLOW);
+    }
+    *ap_out = ap;
+    return n;
+  };
+  // prefix of the lengths over all slots, and the largest one
+  unsigned long long carry = 0, mxl = 0;
   for (int base = 0; base < S; base += blockDim.x) {
     const int s = base + tid;
     unsigned long long x = 0;
     if (s < S) {
-      long long n = max(a.len[s], 0);
-      const long long os = a.off[s];
-      offs[s] = os;
-      const long long room = a.kp_rows - os;
-      if (n > room) { kvc_flag(KVC_DEVERR_INDEX_RANGE); n = room > 0 ? room : 0; }
-      unsigned char ap = 0;
-      if (a.append) {
-        if (a.len[s] >= 0 && n < a.cap[s] && n < room) { ap = 1; ++n; }
-        else if (blockIdx.x == 0) kvc_flag(KVC_DEVERR_APPEND_OVERFLOW);
-      }
+      unsigned char ap;
+      x = (unsigned long long)slot_len(s, &ap, blockIdx.x == 0);
       app[s] = ap;
-      x = (unsigned long long)n;
+      mxl = x > mxl ? x : mxl;
     }
     unsigned long long tot;
     const unsigned long long before = carry + block_exclusive_scan<unsigned long long>(x, scan_sh, &tot);
     if (s < S) P[s] = (long long)before;
     carry += tot;
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(0xffffffffu, mxl, o);
+    mxl = y > mxl ? y : mxl;
+  }
+  if (lane == 0) atomicMax(&max_len_sh, mxl);
+  if (tid == 0) P[S] = (long long)carry;
   if (tid == 0) {
-    P[S] = (long long)carry;
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], C::CONS_WARPS);
@@ -183,14 +225,34 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
 
   const long long N = P[S];
   const int nC = gridDim.x, c = blockIdx.x;
-  for (int s = c; s < S; s += nC)
-    if (P[s + 1] == P[s])
-      for (int e = tid; e < G * D; e += blockDim.x) a.out[(size_t)s * G * D + e] = 0.f;
-  const int nE = (int)min((long long)nC, N);
-  const bool active = N > 0 && c < nE;
-  const long long b0 = active ? (long long)c * N / nE : 0, b1 = active ? (long long)(c + 1) * N / nE : 0;
+  // per-slot clusters: launched in clusters, every slot has one, they fill >= 3/4 of
+  // the grid, and the lengths are near uniform (the same test in every CTA)
+  const bool per_slot = ksz >= 2 && (long long)S * ksz <= nC && 4LL * S * ksz >= 3LL * nC &&
+                       4LL * (long long)max_len_sh * S <= 5LL * N;
+  int nE = 0;
+  bool active = false;
+  long long b0 = 0, b1 = 0;
+  const int my_cluster = c / (ksz > 0 ? ksz : 1);
+  if (!per_slot) {
+    for (int s = c; s < S; s += nC)
+      if (P[s + 1] == P[s])
+        for (int e = tid; e < G * D; e += blockDim.x) a.out[(size_t)s * G * D + e] = 0.f;
+    nE = (int)min((long long)nC, N);
+    active = N > 0 && c < nE;
+    b0 = active ? (long long)c * N / nE : 0;
+    b1 = active ? (long long)(c + 1) * N / nE : 0;
+  } else if (my_cluster < S) {
+    const int sl = my_cluster;
+    const long long r = (long long)cluster_rank(), ns = P[sl + 1] - P[sl];
+    b0 = P[sl] + r * ns / ksz;
+    b1 = P[sl] + (r + 1) * ns / ksz;
+    active = b1 > b0;
+  }
+  if (per_slot)
+    for (int e = tid; e < G * (D + 2); e += blockDim.x) cres[e] = e >= G * D && e < G * D + G ? -INFINITY : 0.f;
 
   auto slot_of = [&](long long t) {
+    if (per_slot) return my_cluster;
     int lo = 0, hi = S - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -421,7 +483,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     }
     named_bar_sync(1, C::CONS_WARPS * 32);
 
-    const int cfirst = cta_of(P[s]), clast = cta_of(P[s + 1] - 1);
+    const int cfirst = per_slot ? 0 : cta_of(P[s]), clast = per_slot ? 0 : cta_of(P[s + 1] - 1);
     const bool single = cfirst == clast;
     float* mypart = a.partial + (size_t)(c + s) * G * (D + 2);
     for (int e = tid; e < G * D; e += C::CONS_WARPS * 32) {
@@ -439,7 +501,13 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         Lt += cmw[G + h] * sc;
         A += cmw[2 * G + e] * sc;
       }
-      if (single) {
+      if (per_slot) {
+        cres[e] = A;
+        if (e % D == 0) {
+          cres[G * D + h] = M;
+          cres[G * D + G + h] = Lt;
+        }
+      } else if (single) {
         a.out[(size_t)s * G * D + e] = Lt > 0.f ? A / Lt : 0.f;
       } else {
         mypart[e] = A;
@@ -449,7 +517,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         }
       }
     }
-    if (!single) {
+    if (!per_slot && !single) {
       // the CTA's partial writes, then one fenced ticket (the barrier + one-thread fence
       // orders every thread's writes before the atomic)
       named_bar_sync(1, C::CONS_WARPS * 32);
@@ -465,6 +533,29 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   }
   }
 
+  if (per_slot) {
+    // every CTA of the slot's cluster has its partial in cres; rank 0 merges them
+    cluster_sync_all();
+    const int k = ksz, sl = my_cluster;
+    if (cluster_rank() == 0 && sl < S) {
+      for (int e = tid; e < G * D; e += blockDim.x) {
+        const int h = e / D;
+        float M = -INFINITY;
+        for (int r = 0; r < k; ++r) M = fmaxf(M, ld_dsmem(cres + G * D + h, r));
+        float Lt = 0.f, A = 0.f;
+        if (M != -INFINITY)
+          for (int r = 0; r < k; ++r) {
+            const float m = ld_dsmem(cres + G * D + h, r);
+            if (m == -INFINITY) continue;
+            const float sc = exp2f(m - M);
+            Lt += ld_dsmem(cres + G * D + G + h, r) * sc;
+            A += ld_dsmem(cres + e, r) * sc;
+          }
+        a.out[(size_t)sl * G * D + e] = Lt > 0.f ? A / Lt : 0.f;
+      }
+    }
+    cluster_sync_all();   // keep every CTA's shared memory alive until rank 0 has read it
+  }
 }
 
 }  // namespace kvc

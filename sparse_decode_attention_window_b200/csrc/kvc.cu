@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <map>
 #include <mutex>
@@ -18,6 +19,7 @@
 #include "select.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "profile.cuh"
 
 namespace {
 
@@ -183,13 +185,74 @@ kvc_status launch_decode(const kvc::DecodeParams& p, int sms, cudaStream_t st) {
   return check_launch("kvc_decode_attn");
 }
 
-// bf16: tensor-core decode (any G <= 8), K/V tiles by TMA through 2-D tensor maps of kp / vp
+// KVC_DECODE_SPLIT=tokens keeps the token-range split even for few slots (cross-checks).
+bool force_token_split() {
+  static const bool v = [] {
+    const char* e = getenv("KVC_DECODE_SPLIT");
+    return e && strcmp(e, "tokens") == 0;
+  }();
+  return v;
+}
+
+// How many clusters of k decode CTAs can be resident at once (shared memory per SM, GPC
+// sizes: a cluster never spans GPCs, so a GPC whose SM count k does not divide leaves SMs
+// idle)? Asked once per (k, device); every decode CTA takes a whole SM's shared memory,
+// so the answer does not depend on the exact size.
 template <int D>
-kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStream_t st) {
+int max_active_clusters(int k, size_t smem, int sms) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> known;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = known.find({k, dev});
+  if (it != known.end()) return it->second;
+  int n = 0;
+  if (set_smem(kvc::decode_mma_kernel<D>, smem, "cluster check") == KVC_OK) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((sms / k) * k);
+    cfg.blockDim = dim3(kvc::DmCfg<D>::THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = k;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kvc::decode_mma_kernel<D>, &cfg) != cudaSuccess) n = 0;
+    cudaGetLastError();
+  }
+  known[{k, dev}] = n;
+  return n;
+}
+
+// bf16: tensor-core decode (any G <= 8), K/V tiles by TMA through 2-D tensor maps of kp / vp.
+// Few slots (2 S <= SMs): clusters of k <= min(8, SMs / S) CTAs, one per slot, when the
+// kernel finds the lengths near uniform; otherwise the token-range split over the grid.
+template <int D>
+kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStream_t st, bool allow_cluster) {
   using namespace kvc;
   DevInfo* di = nullptr;
   if (dev_info(&di) != KVC_OK) return KVC_ERR_CUDA;
+  // cluster size for the per-slot mode (the kernel decides from the lengths whether to
+  // use it). The grid is the resident clusters, at most SMs / k of them; a size is kept
+  // only when the slot-count half of the kernel's test can pass (S k <= grid <= 4/3 S k),
+  // otherwise the launch is a plain one CTA per SM.
+  int k = p.S > 0 ? sms / p.S : 0;
+  if (k > 8) k = 8;
+  if (!allow_cluster || force_token_split()) k = 1;
   const size_t smem = decode_mma_smem_bytes<D>(p.S, G, sms);
+  int grid = sms;
+  for (; k >= 2; k /= 2) {
+    const int n = std::min(sms / k, max_active_clusters<D>(k, smem, sms));
+    const long long g = (long long)n * k, sk = (long long)p.S * k;
+    if (n >= 1 && sk <= g && 4 * sk >= 3 * g) {
+      grid = (int)g;
+      break;
+    }
+  }
+  const bool cluster = k >= 2;
   if (smem > (size_t)di->smem_optin)
     return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: %d slots need %zu B of shared memory (> %d)", p.S, smem,
                 di->smem_optin);
@@ -199,21 +262,25 @@ kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStr
   if (!enc || !make_map_2d_rows(&mk64, enc, p.kp, D, rows, 64) || !make_map_2d_rows(&mk16, enc, p.kp, D, rows, 16) ||
       !make_map_2d_rows(&mv64, enc, p.vp, D, rows, 64) || !make_map_2d_rows(&mv16, enc, p.vp, D, rows, 16))
     return fail(KVC_ERR_CUDA, "kvc_decode_attn: cuTensorMapEncodeTiled failed");
-  kvc_status rc = set_smem(decode_mma_kernel<D>, smem, "kvc_decode_attn");
-  if (rc != KVC_OK) return rc;
   // programmatic dependent launch: this grid may be scheduled while the previous kernel
   // on the stream finishes; the kernel waits (griddepcontrol.wait) before reading inputs
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(sms);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(DmCfg<D>::THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster ? k : 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mma_kernel<D>, mk64, mk16, mv64, mv16, p, G);
+  cfg.numAttrs = cluster ? 2 : 1;
+  kvc_status rc = set_smem(decode_mma_kernel<D>, smem, "kvc_decode_attn");
+  if (rc != KVC_OK) return rc;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mma_kernel<D>, mk64, mk16, mv64, mv16, p, G, cluster ? k : 1);
   if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "kvc_decode_attn: launch: %s", cudaGetErrorString(e));
   count_launches(1);
   return check_launch("kvc_decode_attn");
@@ -230,10 +297,12 @@ kvc_status decode_by_g(int G, const kvc::DecodeParams& p, int sms, cudaStream_t 
 }
 
 // bf16 with G <= 8 -> tensor-core decode; otherwise the CUDA-core decode (G in {1, 2, 4}).
-kvc_status launch_decode_any(const kvc_shape* shape, const kvc::DecodeParams& p, int sms, cudaStream_t stream) {
+// allow_cluster = false keeps the token-range split, whose merge uses the scratch.
+kvc_status launch_decode_any(const kvc_shape* shape, const kvc::DecodeParams& p, int sms, cudaStream_t stream,
+                             bool allow_cluster = true) {
   if (shape->dtype == KVC_BF16 && shape->G <= 8 && !force_simt_decode()) {
-    if (shape->d == 128) return launch_decode_mma<128>(p, shape->G, sms, stream);
-    return launch_decode_mma<64>(p, shape->G, sms, stream);
+    if (shape->d == 128) return launch_decode_mma<128>(p, shape->G, sms, stream, allow_cluster);
+    return launch_decode_mma<64>(p, shape->G, sms, stream, allow_cluster);
   }
   if (shape->dtype == KVC_BF16) {
     if (shape->d == 128) return decode_by_g<__nv_bfloat16, 128>(shape->G, p, sms, stream);
@@ -413,6 +482,7 @@ kvc_status kvc_select(const kvc_shape* shape, const float* score, const int8_t* 
   p.max_sel = max_sel;
   p.count = count;
   p.key_cap = kvc::select_key_cap(shape->L, chunk_end ? C : 0);
+  p.n_local = 0;
   const size_t smem = kvc::select_smem_bytes(p.key_cap);
   if ((rc = set_smem(kvc::select_kernel, smem, "kvc_select")) != KVC_OK) return rc;
   kvc::select_kernel<<<shape->n_slots, kvc::SEL_THREADS, smem, stream>>>(p);
@@ -558,7 +628,7 @@ kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const 
   p.out = out;
   p.partial = reinterpret_cast<float*>(wsb + w.part_off);
   p.counters = reinterpret_cast<int*>(wsb + w.cnt_off);
-  return launch_decode_any(shape, p, di->sms, stream);
+  return launch_decode_any(shape, p, di->sms, stream, /*allow_cluster=*/false);
 }
 
 kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const void* v_new, const void* q, void* kp,
@@ -601,6 +671,63 @@ kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const vo
   p.cap = cap;
   p.len_out = len;
   return launch_decode_any(shape, p, di->sms, stream);
+}
+
+kvc_status kvc_select_chunks(const kvc_shape* shape, const float* chunk_score, const int32_t* chunk_end, int32_t C,
+                             const int32_t* target, int32_t n_local, int32_t* idx, int32_t max_sel, int32_t* count,
+                             cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!chunk_score || !chunk_end || !target || !idx || !count)
+    return fail(KVC_ERR_INVALID_ARG, "kvc_select_chunks: NULL pointer argument");
+  if (C <= 0 || C > shape->L || max_sel <= 0 || n_local < 0)
+    return fail(KVC_ERR_SHAPE, "kvc_select_chunks: need 1 <= C <= L, max_sel > 0, n_local >= 0");
+  // every slot follows the chunk policy; the policy array is not needed
+  kvc::SelectParams p{};
+  p.score = chunk_score;
+  p.policy = nullptr;
+  p.budget = target;
+  p.mass = 0.9f;
+  p.chunk_end = chunk_end;
+  p.C = C;
+  p.L = shape->L;
+  p.n_kv_heads = shape->n_kv_heads;
+  p.batch = shape->batch;
+  p.idx = idx;
+  p.max_sel = max_sel;
+  p.count = count;
+  p.key_cap = kvc::select_key_cap(shape->L, C);
+  p.n_local = n_local;
+  const size_t smem = kvc::select_smem_bytes(p.key_cap);
+  if ((rc = set_smem(kvc::select_kernel, smem, "kvc_select_chunks")) != KVC_OK) return rc;
+  kvc::select_kernel<<<shape->n_slots, kvc::SEL_THREADS, smem, stream>>>(p);
+  count_launches(1);
+  return check_launch("kvc_select_chunks");
+}
+
+kvc_status kvc_retained_mass(const kvc_shape* shape, const float* score, int32_t N, const int32_t* idx,
+                             int32_t max_sel, const int32_t* count, float* retained, cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!score || !idx || !count || !retained) return fail(KVC_ERR_INVALID_ARG, "kvc_retained_mass: NULL pointer");
+  if (N <= 0 || max_sel <= 0) return fail(KVC_ERR_SHAPE, "kvc_retained_mass: N and max_sel must be positive");
+  kvc::retained_mass_kernel<<<shape->n_slots, kvc::PROF_THREADS, 0, stream>>>(score, N, idx, max_sel, count,
+                                                                               retained);
+  count_launches(1);
+  return check_launch("kvc_retained_mass");
+}
+
+kvc_status kvc_profile_heads(const kvc_shape* shape, const float* score, const uint8_t* special_mask,
+                             int32_t window, float tau, int8_t* policy, float* shares, cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!score || !policy) return fail(KVC_ERR_INVALID_ARG, "kvc_profile_heads: score and policy must be non-NULL");
+  if (!(tau > 0.f && tau <= 1.f) || window < 0)
+    return fail(KVC_ERR_INVALID_ARG, "kvc_profile_heads: need 0 < tau <= 1 and window >= 0");
+  kvc::profile_kernel<<<shape->n_slots, kvc::PROF_THREADS, 0, stream>>>(
+      score, shape->L, special_mask, shape->n_kv_heads, shape->batch, window, tau, policy, shares);
+  count_launches(1);
+  return check_launch("kvc_profile_heads");
 }
 
 }  // extern "C"

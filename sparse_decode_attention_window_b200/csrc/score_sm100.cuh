@@ -91,6 +91,8 @@ KVC_DEV float ex2_ftz(float x) {
   return y;
 }
 
+
+
 // Shared-memory matrix descriptor: K-major operand in the 128-byte swizzle layout
 // TMA writes (rows of 128 B, 8-row groups 1024 B apart), start 1024-B aligned.
 KVC_DEV uint64_t smem_desc_sw128(uint32_t saddr) {

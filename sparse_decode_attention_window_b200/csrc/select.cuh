@@ -37,6 +37,7 @@ struct SelectParams {
   int max_sel;
   int32_t* count;
   int key_cap;      // keys the shared-memory cache holds (<= SEL_SMEM_KEYS)
+  int n_local;      // CHUNK: the last n_local chunks are always kept (ChunkLLM local chunks)
 };
 
 KVC_DEV uint32_t order_key(float f) {
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
   uint32_t* keys = reinterpret_cast<uint32_t*>(sel_smem_raw + sizeof(SelShared));
 
   const int s = blockIdx.x;
-  const int pol = a.policy[s];
+  const int pol = a.policy ? a.policy[s] : KVC_POL_CHUNK;   // no policy array: every slot selects chunks
   const int L = a.L;
   int32_t* idx_row = a.idx ? a.idx + (size_t)s * a.max_sel : nullptr;
   const int tid = threadIdx.x;
@@ -124,8 +125,24 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     return;
   }
 
+  // CHUNK with local chunks: the last n_local chunks are kept before any other; giving
+  // them the largest key makes the selection take them first. If they alone reach the
+  // token target, they are the whole selection.
+  const int n_local = chunk ? min(max(a.n_local, 0), N) : 0;
+  if (n_local > 0) {
+    const int first_local_tok = N - n_local > 0 ? ce[N - n_local - 1] + 1 : 0;
+    if ((long long)(L - first_local_tok) >= (long long)a.budget[s]) {
+      emit_range(idx_row, a.max_sel, first_local_tok, L - first_local_tok);
+      if (tid == 0) {
+        if (L - first_local_tok > a.max_sel) kvc_flag(KVC_DEVERR_INDEX_RANGE);
+        a.count[s] = min(L - first_local_tok, a.max_sel);
+      }
+      return;
+    }
+  }
+  auto raw_key = [&](int n) -> uint32_t { return n >= N - n_local ? 0xffffffffu : order_key(sc[n]); };
   if (cached)
-    for (int n = tid; n < N; n += blockDim.x) keys[n] = order_key(sc[n]);
+    for (int n = tid; n < N; n += blockDim.x) keys[n] = raw_key(n);
   // weights
   int fx = 0;
   if (massc) {
@@ -145,7 +162,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     __syncthreads();
     fx = sh.fixed_exp;
   }
-  auto key_of = [&](int n) -> uint32_t { return cached ? keys[n] : order_key(sc[n]); };
+  auto key_of = [&](int n) -> uint32_t { return cached ? keys[n] : raw_key(n); };
   auto weight_of = [&](int n) -> unsigned long long {
     if (chunk) return (unsigned long long)(ce[n] - (n > 0 ? ce[n - 1] : -1));
     if (massc) {

@@ -359,3 +359,102 @@ def test_fused_append_decode_overflow_keeps_old_rows():
     P.check_out(o[G:2 * G], ref1, "bf16", "appended slot")
     assert (o[2 * G:] == 0).all()
     kvc.kvc_get_status()
+
+
+def test_token_split_decode_on_few_slot_workloads():
+    """Workloads with few slots decode through thread-block clusters by default; the
+    token-range split (forced here) passes the same oracle checks."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, KVC_DECODE_SPLIT="tokens")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        "-k", "llama8b_shape_small_context or zigzag_small or chunk_small or fastgen_small "
+                              "or decode_is_independent or separate_append or fused_append_decode_overflow "
+                              "or ragged_context_lengths or gqa_group_sizes"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+# ---------------------------------------------------------------- next rows
+def test_retained_mass_matches_oracle():
+    """Attention retained by the selection (ZigZagKV's attention loss is 0.9 minus it)."""
+    import sparse_decode_attention_window_b200 as kvc
+    wl = get("zigzag").scaled(n_layers=2, L=2048, steps=0)
+    pipe, _ = run_and_check(wl, steps=[])
+    ret = torch.empty(wl.n_slots, dtype=torch.float32, device="cuda")
+    kvc.kvc_retained_mass(pipe.shape, pipe.score, pipe.idx, pipe.count, ret)
+    torch.cuda.synchronize()
+    sc = _np(pipe.score).astype(np.float64)
+    idx, cnt = _np(pipe.idx), _np(pipe.count)
+    for s in range(wl.n_slots):
+        want = O.retained_mass(sc[s], idx[s, :cnt[s]])
+        assert abs(float(ret[s]) - want) <= 1e-6 * max(want, 1e-30) + 1e-7, (s, float(ret[s]), want)
+        assert O.attention_loss(want) >= 0.0
+
+
+def test_profile_heads_matches_oracle():
+    """FastGen-style profiling of each head from its window scores."""
+    import sparse_decode_attention_window_b200 as kvc
+    from sparse_decode_attention_window_b200.pipeline import KvcPipeline
+    from workloads import fastgen_policies
+    wl = get("llama8b").scaled(batch=2, L=3000, top_b=300, steps=0, n_sinks=4)
+    inp = make_inputs(wl, "cuda")
+    pipe = KvcPipeline(wl, inp)
+    pipe.score_step()
+    _, mask = fastgen_policies(wl.scaled(special_frac=0.04))
+    mask = mask.cuda()
+    pol = torch.empty(wl.n_slots, dtype=torch.int8, device="cuda")
+    shares = torch.empty((wl.n_slots, 2), dtype=torch.float32, device="cuda")
+    for tau in (0.05, 0.2, 0.5, 0.99):
+        for W in (64, 256, 2000):
+            kvc.kvc_profile_heads(pipe.shape, pipe.score, pol, W, tau=tau, special_mask=mask, shares=shares)
+            torch.cuda.synchronize()
+            sc = _np(pipe.score).astype(np.float64)
+            got, sh = _np(pol), _np(shares)
+            for s in range(wl.n_slots):
+                b = (s // wl.hkv) % wl.batch
+                want = O.profile_head(sc[s], _np(mask[b]), W, tau)
+                fl = O.retained_mass(sc[s], O.local_indices(wl.L, W))
+                fs = O.retained_mass(sc[s], O.special_indices(_np(mask[b])))
+                assert abs(sh[s, 0] - fl) < 1e-6 and abs(sh[s, 1] - fs) < 1e-6
+                near = min(abs(fl - tau), abs(fs - tau)) < 1e-5
+                assert got[s] == want or near, (s, tau, W, got[s], want, fl, fs)
+
+
+@pytest.mark.parametrize("n_local", [0, 15, 16, 5000])
+def test_chunk_selection_with_local_chunks(n_local):
+    """ChunkLLM selection keeping the most recent chunks, vs the oracle."""
+    import sparse_decode_attention_window_b200 as kvc
+    wl = get("chunk").scaled(L=8000, steps=0)
+    inp = make_inputs(wl, "cpu")
+    from dataclasses import replace
+    dinp = replace(inp, **{f: getattr(inp, f).cuda() for f in ("q_win", "k", "v", "q_dec", "k_dec", "v_dec",
+                                                                 "chunk_end")})
+    from sparse_decode_attention_window_b200.pipeline import KvcPipeline
+    pipe = KvcPipeline(wl, dinp)
+    pipe.score_step()
+    idx = torch.empty((wl.n_slots, wl.L), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(wl.n_slots, dtype=torch.int32, device="cuda")
+    target = torch.full((wl.n_slots,), wl.chunk_target, dtype=torch.int32, device="cuda")
+    kvc.kvc_select_chunks(pipe.shape, pipe.score, dinp.chunk_end, target, idx, cnt, n_local=n_local)
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    ce = _np(dinp.chunk_end)
+    C = len(ce)
+    for s in range(wl.n_slots):
+        ref_sc = O.chunk_scores(inp.q_win[s * wl.G:(s + 1) * wl.G], inp.k[s:s + 1], wl.L, ce)[0]
+        got = _np(idx[s, :int(cnt[s])]).astype(np.int64)
+        toks, chosen = O.chunk_select_local(ref_sc, ce, wl.chunk_target, n_local)
+        if np.array_equal(got, toks):
+            continue
+        # outside exact agreement only the tie band at the cut may differ: the forced chunks and
+        # the clearly-ranked ones must match
+        nl = min(n_local, C)
+        cid = np.unique(np.searchsorted(ce, got, side="left"))
+        assert set(range(C - nl, C)) <= set(cid.tolist())
+        free_sc = ref_sc[: C - nl]
+        P.check_chunks(np.concatenate([np.arange(ce[c - 1] + 1 if c else 0, ce[c] + 1) for c in cid if c < C - nl])
+                       if any(c < C - nl for c in cid) else np.zeros(0, np.int64),
+                       free_sc, ce[: C - nl], wl.chunk_target - int((np.diff(np.concatenate([[-1], ce]))[C - nl:]).sum()),
+                       f"slot {s}")
