@@ -11,6 +11,7 @@
 #include "../../include/kvc.h"
 
 #define KVC_DEV __device__ __forceinline__
+#define KVC_HD __host__ __device__ __forceinline__
 
 // One error word per device (this library is built as a single translation unit).
 __device__ unsigned int g_kvc_deverr;

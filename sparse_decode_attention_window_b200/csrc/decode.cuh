@@ -99,6 +99,10 @@ KVC_DEV void load_part(const unsigned char* row, int p, int rot, float (&f)[D / 
   }
 }
 
+// Floats per (CTA, slot) partial: G*D unnormalised outputs, G maxima, G sums, padded
+// to a multiple of 4 floats so every partial starts 16-byte aligned.
+KVC_HD constexpr int partial_stride(int G, int D) { return (G * (D + 2) + 3) & ~3; }
+
 struct DecodeParams {
   const void* q;
   const void* kp;
@@ -109,7 +113,7 @@ struct DecodeParams {
   int S;
   float scale_log2;
   float* out;
-  float* partial;   // [(gridDim.x + S) * G * (D + 2)]
+  float* partial;   // [(gridDim.x + S) * partial_stride(G, D)]
   int* counters;    // [S + 1], zero on entry and on exit ([S]: grid-wide ticket of the fused append)
   // fused append (tensor-core kernel only): the new token of slot s is k_new[s], v_new[s]
   int append;
@@ -125,7 +129,7 @@ struct DecodeParams {
 // together, so a merge of up to 8 partials costs one round trip to L2.
 KVC_DEV void merge_partials(const DecodeParams& a, int s, int G, int D, int cfirst, int clast, int tid, int nthr) {
   const int np = clast - cfirst + 1;
-  const size_t stride = (size_t)G * (D + 2);
+  const size_t stride = (size_t)partial_stride(G, D);
   const float* base = a.partial + (size_t)(cfirst + s) * stride;
   for (int e = tid; e < G * D; e += nthr) {
     const int h = e / D;
@@ -398,7 +402,7 @@ __global__ void __launch_bounds__(DecCfg<T, D, G>::THREADS, 1) decode_kernel(Dec
 
     const int cfirst = cta_of(P[s]), clast = cta_of(P[s + 1] - 1);
     const bool single = cfirst == clast;
-    float* mypart = a.partial + (size_t)(c + s) * G * (D + 2);
+    float* mypart = a.partial + (size_t)(c + s) * partial_stride(G, D);
     for (int e = tid; e < G * D; e += C::CONS_WARPS * 32) {
       const int h = e / D;
       float M = -INFINITY;

@@ -34,17 +34,49 @@ struct DmCfg {
   static constexpr int STAGE_BYTES = 2 * KB * REGION;
   static constexpr int STAGES = 4;
   static constexpr int CONS_WARPS = 4;               // each consumes one 16-token m-tile per stage
-  static constexpr int THREADS = (CONS_WARPS + 1) * 32;
+  static constexpr int CONS_THREADS = CONS_WARPS * 32;
+  static constexpr int THREADS = CONS_THREADS + 32;
   static constexpr int KSTEPS = D / 16;
   static constexpr int DTILES = D / 16;
+  static constexpr int WO_STRIDE = D + 4;            // padded head row of the in-CTA combine buffer
+};
+
+// Online-softmax rescale threshold (log2 units): a warp keeps its running maximum until
+// a logit exceeds it by more than this, so most tiles skip the max reduction and the
+// rescale; probabilities then stay below 2^8, far inside fp32 and the bf16 hi/lo split.
+constexpr float DM_LAZY_LOG2 = 8.f;
+constexpr int DM_MIN_TOKENS_PER_CTA = 64;            // token split: no CTA gets less than a tile
+constexpr int DM_MAX_CLUSTER = 8;
+
+// Shared-memory layout of decode_mma_kernel (host and device agree on it).
+struct DmLayout {
+  size_t stages, qbuf, bars, P, offs, wm, wo, xr, app, total;
+  template <int D>
+  KVC_HD static DmLayout make(int S, int G, int grid) {
+    using C = DmCfg<D>;
+    DmLayout l{};
+    size_t o = 0;
+    l.stages = o;  o += (size_t)C::STAGES * C::STAGE_BYTES;          // 1024-byte aligned base
+    l.qbuf = o;    o += (size_t)C::STAGES * G * D * 2;               // the segment's q, one per stage
+    l.bars = o;    o += 2 * C::STAGES * sizeof(uint64_t);
+    l.P = o;       o += (size_t)(S + 1) * sizeof(long long);
+    l.offs = o;    o += (size_t)S * sizeof(long long);
+    l.wm = o;      o += 2 * C::CONS_WARPS * 8 * sizeof(float);       // per-warp max and sum, 8 heads
+    l.wo = o;      o += (size_t)C::CONS_WARPS * G * C::WO_STRIDE * sizeof(float);
+    // token split: scale table of the merge [grid][G] + 1/sum [8]; per-slot clusters:
+    // the k CTA records [k][G*D + 2G] that rank 0 merges
+    const size_t tok = ((size_t)grid * G + 8) * sizeof(float);
+    const size_t clu = 2 * S <= grid ? (size_t)DM_MAX_CLUSTER * (G * D + 2 * G) * sizeof(float) : 0;
+    l.xr = o;      o += (tok > clu ? tok : clu);
+    l.app = o;     o += (size_t)S;
+    l.total = o + 1024 + 16;                                          // base alignment slack
+    return l;
+  }
 };
 
 template <int D>
-constexpr size_t decode_mma_smem_bytes(int S, int G, int grid) {
-  using C = DmCfg<D>;
-  return 1024 + (size_t)C::STAGES * C::STAGE_BYTES + 2 * C::STAGES * sizeof(uint64_t) +
-         (size_t)(2 * S + 1) * sizeof(long long) + (size_t)C::CONS_WARPS * (2 * G + G * D) * sizeof(float) +
-         (size_t)2 * grid * G * sizeof(float) + (size_t)G * (D + 2) * sizeof(float) + (size_t)S + 16;
+inline size_t decode_mma_smem_bytes(int S, int G, int grid) {
+  return DmLayout::make<D>(S, G, grid).total;
 }
 
 KVC_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -93,6 +125,15 @@ KVC_DEV float ld_dsmem(const float* local, uint32_t rank) {
   return v;
 }
 
+// Store a float at the same shared-memory offset in CTA `rank` of this cluster.
+KVC_DEV void st_dsmem(float* local, uint32_t rank, float v) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+}
+KVC_DEV void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+KVC_DEV void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
 // Byte offset of (row, 16-byte chunk) in a 128-byte-swizzled region of 128-byte rows.
 KVC_DEV uint32_t swz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
 
@@ -116,15 +157,70 @@ KVC_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
       : "memory");
 }
 
+// The last CTA to finish slot s in the token split merges the slot's CTA partials
+// (CTAs cfirst..clast, stored consecutively at index c + s): warp w finds the maximum
+// and the scaled sum of heads w, w + 4, ... over all partials (lanes stride the
+// partials), then each thread folds float4 columns of the outputs over the partials
+// with independent loads. Runs on the CTA's consumer threads.
+KVC_DEV void merge_partials_par(const DecodeParams& a, int s, int G, int D, int cfirst, int clast, float* sc_tab,
+                                int tid, int nthr) {
+  const int np = clast - cfirst + 1;
+  const size_t stride = (size_t)partial_stride(G, D);
+  const float* base = a.partial + (size_t)(cfirst + s) * stride;
+  float* linv = sc_tab + (size_t)np * G;   // [8]
+  const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+  for (int h = warp; h < G; h += nw) {
+    float M = -INFINITY;
+    for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldcg(base + (size_t)p * stride + (size_t)G * D + h));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Lt = 0.f;
+    for (int p = lane; p < np; p += 32) {
+      const float m = __ldcg(base + (size_t)p * stride + (size_t)G * D + h);
+      const float l = __ldcg(base + (size_t)p * stride + (size_t)G * D + G + h);
+      const float sc = m == -INFINITY ? 0.f : ex2_ftz(m - M);
+      sc_tab[p * G + h] = sc;
+      Lt += l * sc;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lt += __shfl_xor_sync(0xffffffffu, Lt, o);
+    if (lane == 0) linv[h] = Lt > 0.f ? 1.f / Lt : 0.f;
+  }
+  named_bar_sync(1, nthr);
+  const int nq = G * D / 4;
+  for (int c4 = tid; c4 < nq; c4 += nthr) {
+    const int h = (c4 * 4) / D;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int p = 0; p < np; ++p) {
+      const float sc = sc_tab[p * G + h];
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (size_t)p * stride) + c4);
+      acc.x += sc * v.x;
+      acc.y += sc * v.y;
+      acc.z += sc * v.z;
+      acc.w += sc * v.w;
+    }
+    const float li = linv[h];
+    reinterpret_cast<float4*>(a.out + (size_t)s * G * D)[c4] = make_float4(acc.x * li, acc.y * li, acc.z * li, acc.w * li);
+  }
+}
+
 // Two ways to split the work, chosen on the device from the lengths (every CTA reads
 // all of them and reaches the same choice):
 //  * per-slot clusters - when the grid was launched in clusters of k CTAs, every slot
 //    fits one cluster, the clusters cover >= 3/4 of the grid and the lengths are near
 //    uniform (max * S <= 1.25 * total): slot j gets cluster j, whose k CTAs split its
-//    tokens evenly and merge their k partials through distributed shared memory;
-//  * token ranges - otherwise: the valid tokens of all slots are cut into gridDim.x
-//    equal ranges (ranges may cross slots) and partials merge through global tickets.
-template <int D>
+//    tokens evenly; each CTA pushes its record (outputs, max, sum) into rank 0's shared
+//    memory and rank 0 merges the k records after one cluster barrier;
+//  * token ranges - otherwise: the valid tokens of all slots are cut into equal ranges
+//    of at least DM_MIN_TOKENS_PER_CTA (ranges may cross slots); a slot covered by one
+//    CTA is written directly, otherwise partials merge through global tickets.
+// Inside a CTA, warp 4 issues the TMA loads (K and V tiles, and the slot's q with the
+// first tile of a segment) and warps 0-3 each take 16 tokens of every 64-token tile.
+// PACK (G <= 4): the Q^T operand repeats heads 0-3 in columns 4-7, so the same S^T
+// columns 4-7 let the P^T operand carry the bf16 remainder of p next to its bf16 high
+// part, and one O MMA per d-tile accumulates both (summed once per segment).
+template <int D, bool PACK>
 __global__ void __launch_bounds__(DmCfg<D>::THREADS, 1)
 decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constant__ CUtensorMap mk16,
                   const __grid_constant__ CUtensorMap mv64, const __grid_constant__ CUtensorMap mv16,
@@ -133,42 +229,59 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   extern __shared__ __align__(1024) unsigned char dm_raw[];
   const uint32_t raw = smem_u32(dm_raw);
   unsigned char* sm = dm_raw + (((raw + 1023u) & ~1023u) - raw);
-  unsigned char* stages = sm;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::STAGES * C::STAGE_BYTES);
+  const int S = a.S;
+  const DmLayout lay = DmLayout::make<D>(S, G, gridDim.x);
+  unsigned char* stages = sm + lay.stages;
+  unsigned char* qbuf = sm + lay.qbuf;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + lay.bars);
   uint64_t* empty = full + C::STAGES;
-  long long* P = reinterpret_cast<long long*>(empty + C::STAGES);
-  long long* offs = P + a.S + 1;                          // off[] of the slots
-  float* comb = reinterpret_cast<float*>(offs + a.S);    // [warps][2G + G*D]
-  float* cres = comb + C::CONS_WARPS * (2 * G + G * D) + 2 * gridDim.x * G;   // cluster mode: acc[G*D], m[G], l[G]
-  unsigned char* app = reinterpret_cast<unsigned char*>(cres + G * (D + 2));
+  long long* P = reinterpret_cast<long long*>(sm + lay.P);
+  long long* offs = reinterpret_cast<long long*>(sm + lay.offs);
+  float* wm = reinterpret_cast<float*>(sm + lay.wm);        // [warp][8] maxima
+  float* wl = wm + C::CONS_WARPS * 8;                        // [warp][8] sums
+  float* wo = reinterpret_cast<float*>(sm + lay.wo);        // [warp][G][WO_STRIDE]
+  float* xr = reinterpret_cast<float*>(sm + lay.xr);
+  unsigned char* app = sm + lay.app;
   __shared__ unsigned long long scan_sh[33];
   __shared__ int last_flag;
   __shared__ int abort_flag;
   __shared__ unsigned long long max_len_sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) max_len_sh = 0;
-  __syncthreads();
-  const int S = a.S;
-  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
-
-  // Launched with programmatic stream serialization: wait here until the previous
-  // kernel on the stream has completed and its writes are visible (nothing above
-  // reads global memory), then let the next kernel start its own launch.
+  // Nothing before the dependency wait reads global memory that an earlier kernel writes.
+  if (tid == 0) {
+    max_len_sh = 0;
+    abort_flag = 0;
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], C::CONS_WARPS);
+    }
+    fence_mbar_init();
+  }
+  if (warp == C::CONS_WARPS && lane == 0) {
+    prefetch_tensormap(&mk64);
+    prefetch_tensormap(&mv64);
+    prefetch_tensormap(&mk16);
+    prefetch_tensormap(&mv16);
+  }
+  // Launched with programmatic stream serialization: wait until the previous kernel on
+  // the stream has completed and its writes are visible, then let the next one launch.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // One slot's length (clipped to the buffer); with the fused append, a slot that has
   // room gets its new token as its last row.
   auto slot_len = [&](int s, unsigned char* ap_out, bool flag_overflow) -> long long {
-    long long n = max(a.len[s], 0);
+    const int ln = a.len[s];
     const long long os = a.off[s];
+    const int cp = a.append ? a.cap[s] : 0;
+    long long n = max(ln, 0);
     offs[s] = os;
     const long long room = a.kp_rows - os;
     if (n > room) { kvc_flag(KVC_DEVERR_INDEX_RANGE); n = room > 0 ? room : 0; }
     unsigned char ap = 0;
     if (a.append) {
-      if (a.len[s] >= 0 && n < a.cap[s] && n < room) { ap = 1; ++n; }
+      if (ln >= 0 && n < cp && n < room) { ap = 1; ++n; }
       else if (flag_overflow) kvc_flag(KVC_DEVERR_APPEND_OVERFLOW);
     }
     *ap_out = ap;
@@ -197,59 +310,40 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   }
   if (lane == 0) atomicMax(&max_len_sh, mxl);
   if (tid == 0) P[S] = (long long)carry;
-  if (tid == 0) {
-    for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], C::CONS_WARPS);
-    }
-    abort_flag = 0;
-    fence_mbar_init();
-  }
   __syncthreads();
 
-  if (a.append) {
-    // every CTA has read len once its prologue is done; the last CTA to get here
-    // publishes the new lengths (nothing in this launch reads len again)
-    if (tid == 0) {
-      int old;
-      asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(&a.counters[S]), "r"(1) : "memory");
-      last_flag = old == (int)gridDim.x - 1;
-    }
-    __syncthreads();
-    if (last_flag) {
-      for (int s = tid; s < S; s += blockDim.x)
-        if (app[s]) a.len_out[s] = a.len[s] + 1;
-      if (tid == 0) a.counters[S] = 0;
-    }
-  }
+  // Fused append: every CTA has read len once it gets here. Its ticket is taken now but
+  // only looked at when the CTA ends; the CTA that drew the last ticket then publishes
+  // the new lengths (nothing in this launch reads len after its prologue).
+  int ticket = -1;
+  if (a.append && tid == 0)
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(&a.counters[S]), "r"(1) : "memory");
 
   const long long N = P[S];
   const int nC = gridDim.x, c = blockIdx.x;
   // per-slot clusters: launched in clusters, every slot has one, they fill >= 3/4 of
   // the grid, and the lengths are near uniform (the same test in every CTA)
   const bool per_slot = ksz >= 2 && (long long)S * ksz <= nC && 4LL * S * ksz >= 3LL * nC &&
-                       4LL * (long long)max_len_sh * S <= 5LL * N;
+                        4LL * (long long)max_len_sh * S <= 5LL * N;
+  const int my_cluster = c / (ksz > 0 ? ksz : 1);
+  const bool in_slot_cluster = per_slot && my_cluster < S;
   int nE = 0;
   bool active = false;
   long long b0 = 0, b1 = 0;
-  const int my_cluster = c / (ksz > 0 ? ksz : 1);
   if (!per_slot) {
     for (int s = c; s < S; s += nC)
       if (P[s + 1] == P[s])
         for (int e = tid; e < G * D; e += blockDim.x) a.out[(size_t)s * G * D + e] = 0.f;
-    nE = (int)min((long long)nC, N);
+    nE = (int)min((long long)nC, (N + DM_MIN_TOKENS_PER_CTA - 1) / DM_MIN_TOKENS_PER_CTA);
     active = N > 0 && c < nE;
     b0 = active ? (long long)c * N / nE : 0;
     b1 = active ? (long long)(c + 1) * N / nE : 0;
-  } else if (my_cluster < S) {
-    const int sl = my_cluster;
-    const long long r = (long long)cluster_rank(), ns = P[sl + 1] - P[sl];
-    b0 = P[sl] + r * ns / ksz;
-    b1 = P[sl] + (r + 1) * ns / ksz;
+  } else if (in_slot_cluster) {
+    const long long r = (long long)cluster_rank(), ns = P[my_cluster + 1] - P[my_cluster];
+    b0 = P[my_cluster] + r * ns / ksz;
+    b1 = P[my_cluster] + (r + 1) * ns / ksz;
     active = b1 > b0;
   }
-  if (per_slot)
-    for (int e = tid; e < G * (D + 2); e += blockDim.x) cres[e] = e >= G * D && e < G * D + G ? -INFINITY : 0.f;
 
   auto slot_of = [&](long long t) {
     if (per_slot) return my_cluster;
@@ -261,14 +355,12 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     return lo;
   };
   auto cta_of = [&](long long t) { return (int)(((t + 1) * nE - 1) / N); };
+  const uint32_t q_bytes = (uint32_t)(G * D * 2);
 
-  if (!active) {
-    // nothing to stream
-  } else if (warp == C::CONS_WARPS) {
-    // ---------------- producer: TMA of 64-token K and V tiles (16-row boxes for a partial tile)
-    if (lane == 0) {
-      prefetch_tensormap(&mk64);
-      prefetch_tensormap(&mv64);
+  if (warp == C::CONS_WARPS) {
+    // ---------------- producer: TMA of 64-token K and V tiles (16-row boxes for a partial
+    // tile); the first tile of a segment also brings the slot's q
+    if (lane == 0 && active) {
       int stage = 0;
       uint32_t ph = 0;
       long long issued = 0;
@@ -282,8 +374,9 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
           const int row0 = (int)(offs[s] + (u - P[s]));
           unsigned char* kdst = stages + stage * C::STAGE_BYTES;
           unsigned char* vdst = kdst + C::KB * C::REGION;
+          const uint32_t qb = u == t ? q_bytes : 0u;
           if (rows == C::TILE) {
-            mbar_arrive_expect_tx(&full[stage], 2 * C::KB * C::REGION);
+            mbar_arrive_expect_tx(&full[stage], 2 * C::KB * C::REGION + qb);
 #pragma unroll
             for (int kb = 0; kb < C::KB; ++kb) {
               tma_load_2d(kdst + kb * C::REGION, &mk64, kb * 64, row0, &full[stage]);
@@ -291,7 +384,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
             }
           } else {
             const int nbox = (rows + 15) / 16;
-            mbar_arrive_expect_tx(&full[stage], 2 * C::KB * nbox * 16 * 128);
+            mbar_arrive_expect_tx(&full[stage], 2 * C::KB * nbox * 16 * 128 + qb);
             for (int bx = 0; bx < nbox; ++bx)
 #pragma unroll
               for (int kb = 0; kb < C::KB; ++kb) {
@@ -299,6 +392,9 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
                 tma_load_2d(vdst + kb * C::REGION + bx * 16 * 128, &mv16, kb * 64, row0 + bx * 16, &full[stage]);
               }
           }
+          if (qb)
+            bulk_g2s(qbuf + (size_t)stage * q_bytes, static_cast<const unsigned char*>(a.q) + (size_t)s * q_bytes,
+                     q_bytes, &full[stage]);
           ++issued;
           if (++stage == C::STAGES) { stage = 0; ph ^= 1; }
         }
@@ -310,251 +406,302 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         mbar_wait(&full[k % C::STAGES], (uint32_t)((k / C::STAGES) & 1));
     }
     __syncwarp();
-  } else {
-  // ---------------- consumers: warp cw owns rows [16 cw, 16 cw + 16) of every tile
-  const int cw = warp;
-  const int g = lane >> 2, qd = lane & 3;                 // fragment row group, column pair
-  const int h0 = 2 * qd, h1 = 2 * qd + 1;                 // heads of this thread's S^T / O^T columns
-  const int mrow0 = 16 * cw;
-  // ldmatrix lane roles
-  const int lm_j = lane >> 3, lm_r = lane & 7;
-  int stage = 0;
-  uint32_t ph = 0;
-  bool aborted = false;
-  for (long long t = b0; t < b1 && !aborted;) {
-    const int s = slot_of(t);
-    const long long seg_end = min(b1, P[s + 1]);
+  } else if (active || in_slot_cluster) {
+    // ---------------- consumers: warp cw owns rows [16 cw, 16 cw + 16) of every tile
+    const int cw = warp;
+    const int g = lane >> 2, qd = lane & 3;                 // fragment row group, column pair
+    const int mrow0 = 16 * cw;
+    const int lm_j = lane >> 3, lm_r = lane & 7;            // ldmatrix lane roles
+    // heads of this thread's S^T / O^T columns 2qd and 2qd + 1
+    const int hc0 = PACK ? 2 * (qd & 1) : 2 * qd, hc1 = hc0 + 1;
+    const bool lo_cols = PACK && qd >= 2;                   // columns carrying the bf16 remainder
+    const bool own = PACK ? qd < 2 : true;                  // lanes that hold final head values
+    const bool hv0 = own && hc0 < G, hv1 = own && hc1 < G;
+    const int qhead = PACK ? (g & 3) : g;                   // head of Q^T column g
+    int stage = 0;
+    uint32_t ph = 0;
+    bool aborted = false;
+    bool pending_empty = in_slot_cluster && !active;       // a cluster CTA without tokens: one empty record
+    for (long long t = b0; (t < b1 && !aborted) || pending_empty;) {
+      pending_empty = false;
+      const int s = slot_of(t);
+      const long long seg_end = active ? min(b1, P[s + 1]) : t;
 
-    // Q^T operand (k = d, n = head), heads >= G are zero
-    uint32_t qb[C::KSTEPS][2];
-    {
-      const int head = g;
+      uint32_t qb[C::KSTEPS][2];
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+      float o[C::DTILES][4];
 #pragma unroll
-      for (int ks = 0; ks < C::KSTEPS; ++ks) {
-        uint32_t v0 = 0, v1 = 0;
-        if (head < G) {
-          const __nv_bfloat16* qr = q + ((size_t)s * G + head) * D + ks * 16 + 2 * qd;
-          v0 = *reinterpret_cast<const uint32_t*>(qr);
-          v1 = *reinterpret_cast<const uint32_t*>(qr + 8);
-        }
-        qb[ks][0] = v0;
-        qb[ks][1] = v1;
-      }
-    }
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float o[C::DTILES][4];
-#pragma unroll
-    for (int dt = 0; dt < C::DTILES; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+      for (int dt = 0; dt < C::DTILES; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
 
-    for (long long u = t; u < seg_end; u += C::TILE) {
-      const int rows = (int)min((long long)C::TILE, seg_end - u);
-      if (!mbar_wait(&full[stage], ph)) {   // every consumer warp waits on this barrier: all stop here
-        *(volatile int*)&abort_flag = 1;
-        aborted = true;
-        break;
-      }
-      unsigned char* Ks = stages + stage * C::STAGE_BYTES;
-      unsigned char* Vs = Ks + C::KB * C::REGION;
-      const int mv = rows - mrow0;                       // valid rows of this warp's m-tile
-      // fused append: the slot's new token is its last valid row; if it falls in this
-      // warp's m-tile, put it into the staged tile (the cache row is stale) and the cache
-      bool patched = false;
-      if (app[s] && P[s + 1] - 1 >= u && P[s + 1] - 1 < u + rows) {
-        const int tr = (int)(P[s + 1] - 1 - u);
-        if (tr >= mrow0 && tr < mrow0 + 16) {
-          const uint4* kn = static_cast<const uint4*>(a.k_new) + (size_t)s * (D / 8);
-          const uint4* vn = static_cast<const uint4*>(a.v_new) + (size_t)s * (D / 8);
-          const size_t dst_row = (size_t)(offs[s] + (P[s + 1] - 1 - P[s])) * (D / 8);
-          for (int ch = lane; ch < D / 8; ch += 32) {
-            const uint4 kv = kn[ch], vv = vn[ch];
-            *reinterpret_cast<uint4*>(Ks + (ch >> 3) * C::REGION + swz(tr, ch & 7)) = kv;
-            *reinterpret_cast<uint4*>(Vs + (ch >> 3) * C::REGION + swz(tr, ch & 7)) = vv;
-            reinterpret_cast<uint4*>(const_cast<void*>(a.kp))[dst_row + ch] = kv;
-            reinterpret_cast<uint4*>(const_cast<void*>(a.vp))[dst_row + ch] = vv;
-          }
-          patched = true;
-          __syncwarp();
+      for (long long u = t; u < seg_end; u += C::TILE) {
+        const int rows = (int)min((long long)C::TILE, seg_end - u);
+        if (!mbar_wait(&full[stage], ph)) {   // every consumer warp waits on this barrier: all stop here
+          *(volatile int*)&abort_flag = 1;
+          aborted = true;
+          break;
         }
-      }
-      if (mv > 0) {
-        if (mv < 16) {
-          // rows past the segment may hold anything (another slot, unwritten capacity):
-          // zero those V rows so 0 * V stays 0 in the MMA
-          for (int e = lane; e < (16 - mv) * 8 * C::KB; e += 32) {
-            const int rr = mrow0 + mv + e / (8 * C::KB);
-            const int rest = e % (8 * C::KB);
-            *reinterpret_cast<uint4*>(Vs + (rest / 8) * C::REGION + rr * 128 + (rest % 8) * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-          __syncwarp();
-        }
-        // S^T = K_tile . Q^T
-        float cs[4] = {0.f, 0.f, 0.f, 0.f};
-        const int arow = mrow0 + lm_r + 8 * (lm_j & 1);
+        if (u == t) {
+          // Q^T operand (k = d, n = head) from the copy that came with this tile
+          const unsigned char* qs = qbuf + (size_t)stage * q_bytes;
 #pragma unroll
-        for (int ks = 0; ks < C::KSTEPS; ++ks) {
-          const int kb = ks >> 2;
-          const int chunk = (ks & 3) * 2 + (lm_j >> 1);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(smem_u32(Ks + kb * C::REGION + swz(arow, chunk)), a0, a1, a2, a3);
-          mma_bf16(cs, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-        }
-        // tokens t0 = g, t1 = g + 8 of the m-tile; heads h0, h1
-        const bool v0 = g < mv, v1 = g + 8 < mv;
-        const float s00 = v0 ? cs[0] * a.scale_log2 : -INFINITY;   // (t0, h0)
-        const float s01 = v0 ? cs[1] * a.scale_log2 : -INFINITY;   // (t0, h1)
-        const float s10 = v1 ? cs[2] * a.scale_log2 : -INFINITY;   // (t1, h0)
-        const float s11 = v1 ? cs[3] * a.scale_log2 : -INFINITY;   // (t1, h1)
-        float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
-#pragma unroll
-        for (int o_ = 4; o_ < 32; o_ <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
-        }
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        const float al0 = n0 == -INFINITY ? 1.f : exp2f(m0 - n0);
-        const float al1 = n1 == -INFINITY ? 1.f : exp2f(m1 - n1);
-        m0 = n0;
-        m1 = n1;
-        const float p00 = s00 == -INFINITY ? 0.f : exp2f(s00 - n0);
-        const float p01 = s01 == -INFINITY ? 0.f : exp2f(s01 - n1);
-        const float p10 = s10 == -INFINITY ? 0.f : exp2f(s10 - n0);
-        const float p11 = s11 == -INFINITY ? 0.f : exp2f(s11 - n1);
-        l0 = l0 * al0 + p00 + p10;
-        l1 = l1 * al1 + p01 + p11;
-        if (al0 != 1.f || al1 != 1.f) {
-#pragma unroll
-          for (int dt = 0; dt < C::DTILES; ++dt) {
-            o[dt][0] *= al0;
-            o[dt][1] *= al1;
-            o[dt][2] *= al0;
-            o[dt][3] *= al1;
+          for (int ks = 0; ks < C::KSTEPS; ++ks) {
+            uint32_t v0 = 0, v1 = 0;
+            if (qhead < G) {
+              const unsigned char* qr = qs + ((size_t)qhead * D + ks * 16 + 2 * qd) * 2;
+              v0 = *reinterpret_cast<const uint32_t*>(qr);
+              v1 = *reinterpret_cast<const uint32_t*>(qr + 16);
+            }
+            qb[ks][0] = v0;
+            qb[ks][1] = v1;
           }
         }
-        // P^T operand (k = token, n = head): transpose the 8x8 blocks, hi + lo bf16 parts
-        const float r00 = bf16_round(p00), r01 = bf16_round(p01), r10 = bf16_round(p10), r11 = bf16_round(p11);
-        const uint32_t bh0 = movmatrix_t(pack_bf16(r00, r01));
-        const uint32_t bh1 = movmatrix_t(pack_bf16(r10, r11));
-        const uint32_t bl0 = movmatrix_t(pack_bf16(p00 - r00, p01 - r01));
-        const uint32_t bl1 = movmatrix_t(pack_bf16(p10 - r10, p11 - r11));
-        // O^T += V^T . P^T
-        const int vrow = mrow0 + lm_r + 8 * (lm_j >> 1);
-#pragma unroll
-        for (int dt = 0; dt < C::DTILES; ++dt) {
-          const int dcol = dt * 16 + 8 * (lm_j & 1);      // first d of this lane's 8x8 block
-          const int kb = dcol >> 6;
-          const int chunk = (dcol & 63) >> 3;
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(smem_u32(Vs + kb * C::REGION + swz(vrow, chunk)), a0, a1, a2, a3);
-          mma_bf16(o[dt], a0, a1, a2, a3, bh0, bh1);
-          mma_bf16(o[dt], a0, a1, a2, a3, bl0, bl1);
+        unsigned char* Ks = stages + stage * C::STAGE_BYTES;
+        unsigned char* Vs = Ks + C::KB * C::REGION;
+        const int mv = rows - mrow0;                       // valid rows of this warp's m-tile
+        // fused append: the slot's new token is its last valid row; if it falls in this
+        // warp's m-tile, put it into the staged tile (the cache row is stale) and the cache
+        bool patched = false;
+        if (app[s] && P[s + 1] - 1 >= u && P[s + 1] - 1 < u + rows) {
+          const int tr = (int)(P[s + 1] - 1 - u);
+          if (tr >= mrow0 && tr < mrow0 + 16) {
+            const uint4* kn = static_cast<const uint4*>(a.k_new) + (size_t)s * (D / 8);
+            const uint4* vn = static_cast<const uint4*>(a.v_new) + (size_t)s * (D / 8);
+            const size_t dst_row = (size_t)(offs[s] + (P[s + 1] - 1 - P[s])) * (D / 8);
+            for (int ch = lane; ch < D / 8; ch += 32) {
+              const uint4 kv = kn[ch], vv = vn[ch];
+              *reinterpret_cast<uint4*>(Ks + (ch >> 3) * C::REGION + swz(tr, ch & 7)) = kv;
+              *reinterpret_cast<uint4*>(Vs + (ch >> 3) * C::REGION + swz(tr, ch & 7)) = vv;
+              reinterpret_cast<uint4*>(const_cast<void*>(a.kp))[dst_row + ch] = kv;
+              reinterpret_cast<uint4*>(const_cast<void*>(a.vp))[dst_row + ch] = vv;
+            }
+            patched = true;
+            __syncwarp();
+          }
         }
-        if (mv < 16) fence_proxy_async();      // our generic writes precede the next TMA into this stage
+        if (mv > 0) {
+          if (mv < 16) {
+            // rows past the segment may hold anything (another slot, unwritten capacity):
+            // zero those V rows so 0 * V stays 0 in the MMA
+            for (int e = lane; e < (16 - mv) * 8 * C::KB; e += 32) {
+              const int rr = mrow0 + mv + e / (8 * C::KB);
+              const int rest = e % (8 * C::KB);
+              *reinterpret_cast<uint4*>(Vs + (rest / 8) * C::REGION + rr * 128 + (rest % 8) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+            __syncwarp();
+          }
+          // S^T = K_tile . Q^T in four independent accumulators (short dependency chains)
+          float c4[4][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) c4[i][0] = c4[i][1] = c4[i][2] = c4[i][3] = 0.f;
+          const int arow = mrow0 + lm_r + 8 * (lm_j & 1);
+#pragma unroll
+          for (int ks = 0; ks < C::KSTEPS; ++ks) {
+            const int kb = ks >> 2;
+            const int chunk = (ks & 3) * 2 + (lm_j >> 1);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(smem_u32(Ks + kb * C::REGION + swz(arow, chunk)), a0, a1, a2, a3);
+            mma_bf16(c4[ks & 3], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+          }
+          float cs[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) cs[i] = (c4[0][i] + c4[1][i]) + (c4[2][i] + c4[3][i]);
+          // tokens t0 = g, t1 = g + 8 of the m-tile; columns 2qd, 2qd + 1
+          const bool v0 = g < mv, v1 = g + 8 < mv;
+          const float s00 = v0 ? cs[0] * a.scale_log2 : -INFINITY;
+          const float s01 = v0 ? cs[1] * a.scale_log2 : -INFINITY;
+          const float s10 = v1 ? cs[2] * a.scale_log2 : -INFINITY;
+          const float s11 = v1 ? cs[3] * a.scale_log2 : -INFINITY;
+          const bool need = s00 > m0 + DM_LAZY_LOG2 || s10 > m0 + DM_LAZY_LOG2 || s01 > m1 + DM_LAZY_LOG2 ||
+                            s11 > m1 + DM_LAZY_LOG2;
+          if (__any_sync(0xffffffffu, need)) {
+            float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+#pragma unroll
+            for (int o_ = 4; o_ < 32; o_ <<= 1) {
+              mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
+              mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
+            }
+            // row g = 0 of the m-tile is valid, so both maxima are finite here
+            const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+            const float al0 = ex2_ftz(m0 - n0), al1 = ex2_ftz(m1 - n1);   // 0 while m was -inf
+            m0 = n0;
+            m1 = n1;
+            l0 *= al0;
+            l1 *= al1;
+#pragma unroll
+            for (int dt = 0; dt < C::DTILES; ++dt) {
+              o[dt][0] *= al0;
+              o[dt][1] *= al1;
+              o[dt][2] *= al0;
+              o[dt][3] *= al1;
+            }
+          }
+          const float p00 = ex2_ftz(s00 - m0), p01 = ex2_ftz(s01 - m1);   // exp2(-inf) = 0
+          const float p10 = ex2_ftz(s10 - m0), p11 = ex2_ftz(s11 - m1);
+          l0 += p00 + p10;
+          l1 += p01 + p11;
+          // P^T operand (k = token, n = column): transpose the 8x8 blocks with movmatrix
+          const float r00 = bf16_round(p00), r01 = bf16_round(p01), r10 = bf16_round(p10), r11 = bf16_round(p11);
+          const int vrow = mrow0 + lm_r + 8 * (lm_j >> 1);
+          if (PACK) {
+            // pick each lane's values first: movmatrix is a warp-wide .aligned instruction,
+            // so every lane must execute the same one
+            const uint32_t x0 = lo_cols ? pack_bf16(p00 - r00, p01 - r01) : pack_bf16(r00, r01);
+            const uint32_t x1 = lo_cols ? pack_bf16(p10 - r10, p11 - r11) : pack_bf16(r10, r11);
+            const uint32_t b0 = movmatrix_t(x0);
+            const uint32_t b1 = movmatrix_t(x1);
+#pragma unroll
+            for (int dt = 0; dt < C::DTILES; ++dt) {
+              const int dcol = dt * 16 + 8 * (lm_j & 1);
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_t(smem_u32(Vs + (dcol >> 6) * C::REGION + swz(vrow, (dcol & 63) >> 3)), a0, a1, a2, a3);
+              mma_bf16(o[dt], a0, a1, a2, a3, b0, b1);
+            }
+          } else {
+            const uint32_t bh0 = movmatrix_t(pack_bf16(r00, r01));
+            const uint32_t bh1 = movmatrix_t(pack_bf16(r10, r11));
+            const uint32_t bl0 = movmatrix_t(pack_bf16(p00 - r00, p01 - r01));
+            const uint32_t bl1 = movmatrix_t(pack_bf16(p10 - r10, p11 - r11));
+#pragma unroll
+            for (int dt = 0; dt < C::DTILES; ++dt) {
+              const int dcol = dt * 16 + 8 * (lm_j & 1);
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_t(smem_u32(Vs + (dcol >> 6) * C::REGION + swz(vrow, (dcol & 63) >> 3)), a0, a1, a2, a3);
+              mma_bf16(o[dt], a0, a1, a2, a3, bh0, bh1);
+              mma_bf16(o[dt], a0, a1, a2, a3, bl0, bl1);
+            }
+          }
+          if (mv < 16) fence_proxy_async();      // our generic writes precede the next TMA into this stage
+        }
+        if (patched) fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == C::STAGES) { stage = 0; ph ^= 1; }
       }
-      if (patched) fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[stage]);
-      if (++stage == C::STAGES) { stage = 0; ph ^= 1; }
-    }
+      if (aborted) break;
 
-    if (aborted) break;
-    // ---- per-warp totals: l over the 8 token rows of the fragment
+      // ---- the warp's totals: l over its 8 row groups; PACK adds the remainder columns
 #pragma unroll
-    for (int o_ = 4; o_ < 32; o_ <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, o_);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, o_);
-    }
-    float* cm = comb + cw * (2 * G + G * D);   // m[G], l[G], acc[G][D]
-    if (g == 0) {
-      if (h0 < G) { cm[h0] = m0; cm[G + h0] = l0; }
-      if (h1 < G) { cm[h1] = m1; cm[G + h1] = l1; }
-    }
-#pragma unroll
-    for (int dt = 0; dt < C::DTILES; ++dt) {
-      const int d0 = dt * 16 + g;
-      if (h0 < G) {
-        cm[2 * G + h0 * D + d0] = o[dt][0];
-        cm[2 * G + h0 * D + d0 + 8] = o[dt][2];
+      for (int o_ = 4; o_ < 32; o_ <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o_);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o_);
       }
-      if (h1 < G) {
-        cm[2 * G + h1 * D + d0] = o[dt][1];
-        cm[2 * G + h1 * D + d0 + 8] = o[dt][3];
-      }
-    }
-    named_bar_sync(1, C::CONS_WARPS * 32);
-
-    const int cfirst = per_slot ? 0 : cta_of(P[s]), clast = per_slot ? 0 : cta_of(P[s + 1] - 1);
-    const bool single = cfirst == clast;
-    float* mypart = a.partial + (size_t)(c + s) * G * (D + 2);
-    for (int e = tid; e < G * D; e += C::CONS_WARPS * 32) {
-      const int h = e / D;
-      float M = -INFINITY;
+      if (PACK) {
 #pragma unroll
-      for (int w = 0; w < C::CONS_WARPS; ++w) M = fmaxf(M, comb[w * (2 * G + G * D) + h]);
-      float Lt = 0.f, A = 0.f;
+        for (int dt = 0; dt < C::DTILES; ++dt)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) o[dt][j] += __shfl_down_sync(0xffffffffu, o[dt][j], 2, 4);
+      }
+      // ---- combine the 4 warps: common maximum per head, scaled sums
+      if (g == 0) {
+        if (hv0) wm[cw * 8 + hc0] = m0;
+        if (hv1) wm[cw * 8 + hc1] = m1;
+      }
+      named_bar_sync(1, C::CONS_THREADS);
+      float M0 = -INFINITY, M1 = -INFINITY;
 #pragma unroll
       for (int w = 0; w < C::CONS_WARPS; ++w) {
-        const float* cmw = comb + w * (2 * G + G * D);
-        const float mw = cmw[h];
-        if (mw == -INFINITY) continue;
-        const float sc = exp2f(mw - M);
-        Lt += cmw[G + h] * sc;
-        A += cmw[2 * G + e] * sc;
+        if (hv0) M0 = fmaxf(M0, wm[w * 8 + hc0]);
+        if (hv1) M1 = fmaxf(M1, wm[w * 8 + hc1]);
       }
-      if (per_slot) {
-        cres[e] = A;
-        if (e % D == 0) {
-          cres[G * D + h] = M;
-          cres[G * D + G + h] = Lt;
+      const float f0 = m0 == -INFINITY ? 0.f : ex2_ftz(m0 - M0);
+      const float f1 = m1 == -INFINITY ? 0.f : ex2_ftz(m1 - M1);
+      float* wow = wo + (size_t)cw * G * C::WO_STRIDE;
+#pragma unroll
+      for (int dt = 0; dt < C::DTILES; ++dt) {
+        const int d0 = dt * 16 + g;
+        if (hv0) {
+          wow[hc0 * C::WO_STRIDE + d0] = o[dt][0] * f0;
+          wow[hc0 * C::WO_STRIDE + d0 + 8] = o[dt][2] * f0;
         }
-      } else if (single) {
-        a.out[(size_t)s * G * D + e] = Lt > 0.f ? A / Lt : 0.f;
-      } else {
-        mypart[e] = A;
-        if (e % D == 0) {
-          mypart[G * D + h] = M;
-          mypart[G * D + G + h] = Lt;
+        if (hv1) {
+          wow[hc1 * C::WO_STRIDE + d0] = o[dt][1] * f1;
+          wow[hc1 * C::WO_STRIDE + d0 + 8] = o[dt][3] * f1;
         }
       }
-    }
-    if (!per_slot && !single) {
-      // the CTA's partial writes, then one fenced ticket (the barrier + one-thread fence
-      // orders every thread's writes before the atomic)
-      named_bar_sync(1, C::CONS_WARPS * 32);
-      if (tid == 0) last_flag = slot_ticket(&a.counters[s], clast - cfirst);
-      named_bar_sync(1, C::CONS_WARPS * 32);
-      if (last_flag) {
-        merge_partials(a, s, G, D, cfirst, clast, tid, C::CONS_WARPS * 32);
-        if (tid == 0) a.counters[s] = 0;
+      if (g == 0) {
+        if (hv0) wl[cw * 8 + hc0] = l0 * f0;
+        if (hv1) wl[cw * 8 + hc1] = l1 * f1;
       }
+      named_bar_sync(1, C::CONS_THREADS);
+
+      const int cfirst = per_slot ? 0 : cta_of(P[s]), clast = per_slot ? 0 : cta_of(P[s + 1] - 1);
+      const bool single = !per_slot && cfirst == clast;
+      float* mypart = a.partial + (size_t)(c + s) * partial_stride(G, D);
+      const uint32_t my_rank = per_slot ? cluster_rank() : 0u;
+      float* rec = xr + (size_t)my_rank * (G * D + 2 * G);   // this CTA's record in rank 0's memory
+      for (int e = tid; e < G * D; e += C::CONS_THREADS) {
+        const int h = e / D, d = e - h * D;
+        float A = 0.f, Mh = -INFINITY, Lh = 0.f;
+#pragma unroll
+        for (int w = 0; w < C::CONS_WARPS; ++w) {
+          A += wo[((size_t)w * G + h) * C::WO_STRIDE + d];
+          Mh = fmaxf(Mh, wm[w * 8 + h]);
+          Lh += wl[w * 8 + h];
+        }
+        if (per_slot) {
+          st_dsmem(rec + e, 0, A);
+          if (d == 0) {
+            st_dsmem(rec + G * D + h, 0, Mh);
+            st_dsmem(rec + G * D + G + h, 0, Lh);
+          }
+        } else if (single) {
+          a.out[(size_t)s * G * D + e] = Lh > 0.f ? A / Lh : 0.f;
+        } else {
+          mypart[e] = A;
+          if (d == 0) {
+            mypart[G * D + h] = Mh;
+            mypart[G * D + G + h] = Lh;
+          }
+        }
+      }
+      if (!per_slot && !single) {
+        // the CTA's partial writes, then one fenced ticket (the barrier + one-thread fence
+        // orders every thread's writes before the atomic)
+        named_bar_sync(1, C::CONS_THREADS);
+        if (tid == 0) last_flag = slot_ticket(&a.counters[s], clast - cfirst);
+        named_bar_sync(1, C::CONS_THREADS);
+        if (last_flag) {
+          merge_partials_par(a, s, G, D, cfirst, clast, xr, tid, C::CONS_THREADS);
+          if (tid == 0) a.counters[s] = 0;
+        }
+      }
+      named_bar_sync(1, C::CONS_THREADS);   // wm / wo / xr are reused by the next segment
+      t = seg_end;
     }
-    named_bar_sync(1, C::CONS_WARPS * 32);
-    t = seg_end;
-  }
   }
 
-  if (per_slot) {
-    // every CTA of the slot's cluster has its partial in cres; rank 0 merges them
-    cluster_sync_all();
-    const int k = ksz, sl = my_cluster;
-    if (cluster_rank() == 0 && sl < S) {
+  if (in_slot_cluster) {
+    // every CTA of the slot's cluster has pushed its record; rank 0 merges them
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    if (cluster_rank() == 0) {
+      const int rs = G * D + 2 * G;
       for (int e = tid; e < G * D; e += blockDim.x) {
         const int h = e / D;
         float M = -INFINITY;
-        for (int r = 0; r < k; ++r) M = fmaxf(M, ld_dsmem(cres + G * D + h, r));
+        for (int r = 0; r < ksz; ++r) M = fmaxf(M, xr[r * rs + G * D + h]);
         float Lt = 0.f, A = 0.f;
         if (M != -INFINITY)
-          for (int r = 0; r < k; ++r) {
-            const float m = ld_dsmem(cres + G * D + h, r);
-            if (m == -INFINITY) continue;
-            const float sc = exp2f(m - M);
-            Lt += ld_dsmem(cres + G * D + G + h, r) * sc;
-            A += ld_dsmem(cres + e, r) * sc;
+          for (int r = 0; r < ksz; ++r) {
+            const float m = xr[r * rs + G * D + h];
+            const float sc = m == -INFINITY ? 0.f : ex2_ftz(m - M);
+            Lt += xr[r * rs + G * D + G + h] * sc;
+            A += xr[r * rs + e] * sc;
           }
-        a.out[(size_t)sl * G * D + e] = Lt > 0.f ? A / Lt : 0.f;
+        a.out[(size_t)my_cluster * G * D + e] = Lt > 0.f ? A / Lt : 0.f;
       }
     }
-    cluster_sync_all();   // keep every CTA's shared memory alive until rank 0 has read it
+  }
+
+  if (a.append) {
+    if (tid == 0) last_flag = ticket == (int)gridDim.x - 1;
+    __syncthreads();
+    if (last_flag) {
+      for (int s = tid; s < S; s += blockDim.x)
+        if (app[s]) a.len_out[s] = a.len[s] + 1;
+      if (tid == 0) a.counters[S] = 0;
+    }
   }
 }
 

@@ -163,7 +163,7 @@ DecodeWs decode_ws_layout(const kvc_shape* sh, int sms) {
   w.cnt_off = 0;
   w.cnt_bytes = align_up((size_t)(sh->n_slots + 1) * sizeof(int), 256);
   w.part_off = w.cnt_bytes;
-  w.part_bytes = align_up((size_t)(sms + sh->n_slots) * sh->G * (sh->d + 2) * sizeof(float), 256);
+  w.part_bytes = align_up((size_t)(sms + sh->n_slots) * kvc::partial_stride(sh->G, sh->d) * sizeof(float), 256);
   w.total = w.part_off + w.part_bytes;
   return w;
 }
@@ -198,7 +198,7 @@ bool force_token_split() {
 // sizes: a cluster never spans GPCs, so a GPC whose SM count k does not divide leaves SMs
 // idle)? Asked once per (k, device); every decode CTA takes a whole SM's shared memory,
 // so the answer does not depend on the exact size.
-template <int D>
+template <int D, bool PACK>
 int max_active_clusters(int k, size_t smem, int sms) {
   static std::mutex mu;
   static std::map<std::pair<int, int>, int> known;
@@ -208,7 +208,7 @@ int max_active_clusters(int k, size_t smem, int sms) {
   auto it = known.find({k, dev});
   if (it != known.end()) return it->second;
   int n = 0;
-  if (set_smem(kvc::decode_mma_kernel<D>, smem, "cluster check") == KVC_OK) {
+  if (set_smem(kvc::decode_mma_kernel<D, PACK>, smem, "cluster check") == KVC_OK) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((sms / k) * k);
     cfg.blockDim = dim3(kvc::DmCfg<D>::THREADS);
@@ -220,7 +220,7 @@ int max_active_clusters(int k, size_t smem, int sms) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&n, kvc::decode_mma_kernel<D>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kvc::decode_mma_kernel<D, PACK>, &cfg) != cudaSuccess) n = 0;
     cudaGetLastError();
   }
   known[{k, dev}] = n;
@@ -230,7 +230,7 @@ int max_active_clusters(int k, size_t smem, int sms) {
 // bf16: tensor-core decode (any G <= 8), K/V tiles by TMA through 2-D tensor maps of kp / vp.
 // Few slots (2 S <= SMs): clusters of k <= min(8, SMs / S) CTAs, one per slot, when the
 // kernel finds the lengths near uniform; otherwise the token-range split over the grid.
-template <int D>
+template <int D, bool PACK>
 kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStream_t st, bool allow_cluster) {
   using namespace kvc;
   DevInfo* di = nullptr;
@@ -240,12 +240,15 @@ kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStr
   // only when the slot-count half of the kernel's test can pass (S k <= grid <= 4/3 S k),
   // otherwise the launch is a plain one CTA per SM.
   int k = p.S > 0 ? sms / p.S : 0;
-  if (k > 8) k = 8;
+  if (k > DM_MAX_CLUSTER) k = DM_MAX_CLUSTER;
   if (!allow_cluster || force_token_split()) k = 1;
-  const size_t smem = decode_mma_smem_bytes<D>(p.S, G, sms);
+  const size_t smem_max = decode_mma_smem_bytes<D>(p.S, G, sms);   // any grid <= SMs fits in this
+  if (smem_max > (size_t)di->smem_optin)
+    return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: %d slots need %zu B of shared memory (> %d)", p.S, smem_max,
+                di->smem_optin);
   int grid = sms;
   for (; k >= 2; k /= 2) {
-    const int n = std::min(sms / k, max_active_clusters<D>(k, smem, sms));
+    const int n = std::min(sms / k, max_active_clusters<D, PACK>(k, smem_max, sms));
     const long long g = (long long)n * k, sk = (long long)p.S * k;
     if (n >= 1 && sk <= g && 4 * sk >= 3 * g) {
       grid = (int)g;
@@ -253,9 +256,7 @@ kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStr
     }
   }
   const bool cluster = k >= 2;
-  if (smem > (size_t)di->smem_optin)
-    return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: %d slots need %zu B of shared memory (> %d)", p.S, smem,
-                di->smem_optin);
+  const size_t smem = decode_mma_smem_bytes<D>(p.S, G, grid);
   encode_tiled_fn enc = get_encode_tiled();
   CUtensorMap mk64, mk16, mv64, mv16;
   const long long rows = p.kp_rows > 0 ? p.kp_rows : 1;
@@ -278,9 +279,9 @@ kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStr
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = cluster ? 2 : 1;
-  kvc_status rc = set_smem(decode_mma_kernel<D>, smem, "kvc_decode_attn");
+  kvc_status rc = set_smem(decode_mma_kernel<D, PACK>, smem_max, "kvc_decode_attn");
   if (rc != KVC_OK) return rc;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mma_kernel<D>, mk64, mk16, mv64, mv16, p, G, cluster ? k : 1);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mma_kernel<D, PACK>, mk64, mk16, mv64, mv16, p, G, cluster ? k : 1);
   if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "kvc_decode_attn: launch: %s", cudaGetErrorString(e));
   count_launches(1);
   return check_launch("kvc_decode_attn");
@@ -301,8 +302,12 @@ kvc_status decode_by_g(int G, const kvc::DecodeParams& p, int sms, cudaStream_t 
 kvc_status launch_decode_any(const kvc_shape* shape, const kvc::DecodeParams& p, int sms, cudaStream_t stream,
                              bool allow_cluster = true) {
   if (shape->dtype == KVC_BF16 && shape->G <= 8 && !force_simt_decode()) {
-    if (shape->d == 128) return launch_decode_mma<128>(p, shape->G, sms, stream, allow_cluster);
-    return launch_decode_mma<64>(p, shape->G, sms, stream, allow_cluster);
+    const bool pack = shape->G <= 4;   // heads and the bf16 remainder share one MMA
+    if (shape->d == 128)
+      return pack ? launch_decode_mma<128, true>(p, shape->G, sms, stream, allow_cluster)
+                  : launch_decode_mma<128, false>(p, shape->G, sms, stream, allow_cluster);
+    return pack ? launch_decode_mma<64, true>(p, shape->G, sms, stream, allow_cluster)
+                : launch_decode_mma<64, false>(p, shape->G, sms, stream, allow_cluster);
   }
   if (shape->dtype == KVC_BF16) {
     if (shape->d == 128) return decode_by_g<__nv_bfloat16, 128>(shape->G, p, sms, stream);
@@ -567,8 +572,8 @@ kvc_status kvc_decode_attn(const kvc_shape* shape, const void* q, const void* kp
   if (!q || !kp || !vp || !off || !len || !out) return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn: NULL pointer argument");
   if (shape->n_slots > kvc::DEC_MAX_SLOTS)
     return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: %d slots > %d", shape->n_slots, kvc::DEC_MAX_SLOTS);
-  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(ws))
-    return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn: q, kp, vp, ws must be 16-byte aligned");
+  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(ws) || !aligned16(out))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn: q, kp, vp, out, ws must be 16-byte aligned");
   DevInfo* di = nullptr;
   if ((rc = dev_info(&di)) != KVC_OK) return rc;
   const DecodeWs w = decode_ws_layout(shape, di->sms);
@@ -601,8 +606,8 @@ kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const 
     return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn_noalloc: NULL pointer argument");
   if (shape->n_slots > kvc::DEC_MAX_SLOTS)
     return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn_noalloc: %d slots > %d", shape->n_slots, kvc::DEC_MAX_SLOTS);
-  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp))
-    return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn_noalloc: q, kp, vp must be 16-byte aligned");
+  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(out))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_decode_attn_noalloc: q, kp, vp, out must be 16-byte aligned");
   DevInfo* di = nullptr;
   if ((rc = dev_info(&di)) != KVC_OK) return rc;
   const DecodeWs w = decode_ws_layout(shape, di->sms);
@@ -645,7 +650,8 @@ kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const vo
   }
   if (shape->n_slots > kvc::DEC_MAX_SLOTS)
     return fail(KVC_ERR_UNSUPPORTED, "kvc_append_decode: %d slots > %d", shape->n_slots, kvc::DEC_MAX_SLOTS);
-  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(ws) || !aligned16(k_new) || !aligned16(v_new))
+  if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(ws) || !aligned16(k_new) || !aligned16(v_new) ||
+      !aligned16(out))
     return fail(KVC_ERR_INVALID_ARG, "kvc_append_decode: buffers must be 16-byte aligned");
   DevInfo* di = nullptr;
   if ((rc = dev_info(&di)) != KVC_OK) return rc;
