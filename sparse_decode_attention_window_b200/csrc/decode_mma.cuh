@@ -58,7 +58,7 @@ struct DmLayout {
     size_t o = 0;
     l.stages = o;  o += (size_t)C::STAGES * C::STAGE_BYTES;          // 1024-byte aligned base
     l.qbuf = o;    o += (size_t)C::STAGES * G * D * 2;               // the segment's q, one per stage
-    l.bars = o;    o += 2 * C::STAGES * sizeof(uint64_t);
+    l.bars = o;    o += (2 * C::STAGES + 1) * sizeof(uint64_t);      // full, empty, rank 0's record barrier
     l.P = o;       o += (size_t)(S + 1) * sizeof(long long);
     l.offs = o;    o += (size_t)S * sizeof(long long);
     l.wm = o;      o += 2 * C::CONS_WARPS * 8 * sizeof(float);       // per-warp max and sum, 8 heads
@@ -66,7 +66,7 @@ struct DmLayout {
     // token split: scale table of the merge [grid][G] + 1/sum [8]; per-slot clusters:
     // the k CTA records [k][G*D + 2G] that rank 0 merges
     const size_t tok = ((size_t)grid * G + 8) * sizeof(float);
-    const size_t clu = 2 * S <= grid ? (size_t)DM_MAX_CLUSTER * (G * D + 2 * G) * sizeof(float) : 0;
+    const size_t clu = 2 * S <= grid ? (size_t)DM_MAX_CLUSTER * partial_stride(G, D) * sizeof(float) : 0;
     l.xr = o;      o += (tok > clu ? tok : clu);
     l.app = o;     o += (size_t)S;
     l.total = o + 1024 + 16;                                          // base alignment slack
@@ -108,31 +108,54 @@ KVC_DEV uint32_t pack_bf16(float lo, float hi) {
 }
 KVC_DEV float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
-KVC_DEV void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 KVC_DEV uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
-// Read a float from the same shared-memory offset in CTA `rank` of this cluster.
-KVC_DEV float ld_dsmem(const float* local, uint32_t rank) {
-  uint32_t ra;
-  float v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
-  return v;
-}
 
-// Store a float at the same shared-memory offset in CTA `rank` of this cluster.
-KVC_DEV void st_dsmem(float* local, uint32_t rank, float v) {
+
+// Map a local shared-memory address to the same offset in CTA `rank` of the cluster.
+KVC_DEV uint32_t map_to_rank(const void* local, uint32_t rank) {
   uint32_t ra;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
+  return ra;
 }
-KVC_DEV void cluster_arrive_release() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
-KVC_DEV void cluster_wait_acquire() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// Asynchronous 4-byte store into another CTA's shared memory; its completion counts 4
+// bytes on that CTA's mbarrier.
+KVC_DEV void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+KVC_DEV void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
+KVC_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// Bounded wait with cluster-scope acquire (data that other CTAs sent with st.async).
+KVC_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  auto try_once = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (try_once()) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (try_once()) return true;
+    if (global_timer_ns() - t0 > KVC_WAIT_LIMIT_NS) {
+      kvc_flag(KVC_DEVERR_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
 
 // Byte offset of (row, 16-byte chunk) in a 128-byte-swizzled region of 128-byte rows.
 KVC_DEV uint32_t swz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
@@ -235,6 +258,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   unsigned char* qbuf = sm + lay.qbuf;
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + lay.bars);
   uint64_t* empty = full + C::STAGES;
+  uint64_t* rec_bar = empty + C::STAGES;   // rank 0 of a slot cluster: the other CTAs' records (st.async bytes)
   long long* P = reinterpret_cast<long long*>(sm + lay.P);
   long long* offs = reinterpret_cast<long long*>(sm + lay.offs);
   float* wm = reinterpret_cast<float*>(sm + lay.wm);        // [warp][8] maxima
@@ -256,6 +280,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], C::CONS_WARPS);
     }
+    mbar_init(rec_bar, 1);
     fence_mbar_init();
   }
   if (warp == C::CONS_WARPS && lane == 0) {
@@ -264,6 +289,10 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     prefetch_tensormap(&mk16);
     prefetch_tensormap(&mv16);
   }
+  // cluster launch: every CTA's barrier initialisation is visible cluster-wide before
+  // any CTA sends to another (the matching wait comes before the first st.async)
+  if (ksz >= 2) cluster_arrive_relaxed();
+  bool cl_waited = false;
   // Launched with programmatic stream serialization: wait until the previous kernel on
   // the stream has completed and its writes are visible, then let the next one launch.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -370,7 +399,11 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         const long long seg_end = min(b1, P[s + 1]);
         for (long long u = t; u < seg_end; u += C::TILE) {
           const int rows = (int)min((long long)C::TILE, seg_end - u);
-          if (!mbar_wait(&empty[stage], ph ^ 1) || *(volatile int*)&abort_flag) { ok = false; break; }
+          // the first STAGES tiles find their stages free
+          if ((issued >= C::STAGES && !mbar_wait(&empty[stage], ph ^ 1)) || *(volatile int*)&abort_flag) {
+            ok = false;
+            break;
+          }
           const int row0 = (int)(offs[s] + (u - P[s]));
           unsigned char* kdst = stages + stage * C::STAGE_BYTES;
           unsigned char* vdst = kdst + C::KB * C::REGION;
@@ -629,7 +662,18 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       const bool single = !per_slot && cfirst == clast;
       float* mypart = a.partial + (size_t)(c + s) * partial_stride(G, D);
       const uint32_t my_rank = per_slot ? cluster_rank() : 0u;
-      float* rec = xr + (size_t)my_rank * (G * D + 2 * G);   // this CTA's record in rank 0's memory
+      float* rec = xr + (size_t)my_rank * partial_stride(G, D);   // this CTA's record in rank 0's memory
+      uint32_t rec_remote = 0, bar_remote = 0;
+      if (per_slot) {
+        // rank 0's barrier is initialised (cluster-wide arrive at the start); the record goes
+        // there by st.async, counted on rank 0's record barrier
+        cluster_wait();
+        cl_waited = true;
+        if (my_rank != 0) {
+          rec_remote = map_to_rank(rec, 0);
+          bar_remote = map_to_rank(rec_bar, 0);
+        }
+      }
       for (int e = tid; e < G * D; e += C::CONS_THREADS) {
         const int h = e / D, d = e - h * D;
         float A = 0.f, Mh = -INFINITY, Lh = 0.f;
@@ -639,11 +683,17 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
           Mh = fmaxf(Mh, wm[w * 8 + h]);
           Lh += wl[w * 8 + h];
         }
-        if (per_slot) {
-          st_dsmem(rec + e, 0, A);
+        if (per_slot && my_rank == 0) {
+          rec[e] = A;
           if (d == 0) {
-            st_dsmem(rec + G * D + h, 0, Mh);
-            st_dsmem(rec + G * D + G + h, 0, Lh);
+            rec[G * D + h] = Mh;
+            rec[G * D + G + h] = Lh;
+          }
+        } else if (per_slot) {
+          st_async_f32(rec_remote + 4u * (uint32_t)e, A, bar_remote);
+          if (d == 0) {
+            st_async_f32(rec_remote + 4u * (uint32_t)(G * D + h), Mh, bar_remote);
+            st_async_f32(rec_remote + 4u * (uint32_t)(G * D + G + h), Lh, bar_remote);
           }
         } else if (single) {
           a.out[(size_t)s * G * D + e] = Lh > 0.f ? A / Lh : 0.f;
@@ -669,30 +719,38 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       named_bar_sync(1, C::CONS_THREADS);   // wm / wo / xr are reused by the next segment
       t = seg_end;
     }
-  }
 
-  if (in_slot_cluster) {
-    // every CTA of the slot's cluster has pushed its record; rank 0 merges them
-    cluster_arrive_release();
-    cluster_wait_acquire();
-    if (cluster_rank() == 0) {
-      const int rs = G * D + 2 * G;
-      for (int e = tid; e < G * D; e += blockDim.x) {
-        const int h = e / D;
-        float M = -INFINITY;
-        for (int r = 0; r < ksz; ++r) M = fmaxf(M, xr[r * rs + G * D + h]);
-        float Lt = 0.f, A = 0.f;
-        if (M != -INFINITY)
+    if (in_slot_cluster && !aborted && cluster_rank() == 0) {
+      // rank 0: its own record is in place; wait for the other ksz - 1, then merge
+      const int rs = partial_stride(G, D);
+      if (tid == 0) mbar_arrive_expect_tx(rec_bar, (uint32_t)((ksz - 1) * (G * D + 2 * G) * 4));
+      if (mbar_wait_cluster(rec_bar, 0)) {
+        float* sc = wo;              // [ksz][8] weights, then 1 / sum [8] (the combine buffer is free)
+        float* linv = sc + 8 * 8;
+        if (tid < G) {
+          float M = -INFINITY;
+          for (int r = 0; r < ksz; ++r) M = fmaxf(M, xr[r * rs + G * D + tid]);
+          float Lt = 0.f;
           for (int r = 0; r < ksz; ++r) {
-            const float m = xr[r * rs + G * D + h];
-            const float sc = m == -INFINITY ? 0.f : ex2_ftz(m - M);
-            Lt += xr[r * rs + G * D + G + h] * sc;
-            A += xr[r * rs + e] * sc;
+            const float mr = xr[r * rs + G * D + tid];
+            const float w = mr == -INFINITY ? 0.f : ex2_ftz(mr - M);
+            sc[r * 8 + tid] = w;
+            Lt += xr[r * rs + G * D + G + tid] * w;
           }
-        a.out[(size_t)my_cluster * G * D + e] = Lt > 0.f ? A / Lt : 0.f;
+          linv[tid] = Lt > 0.f ? 1.f / Lt : 0.f;
+        }
+        named_bar_sync(1, C::CONS_THREADS);
+        for (int e = tid; e < G * D; e += C::CONS_THREADS) {
+          const int h = e / D;
+          float acc = 0.f;
+          for (int r = 0; r < ksz; ++r) acc += sc[r * 8 + h] * xr[r * rs + e];
+          a.out[(size_t)my_cluster * G * D + e] = acc * linv[h];
+        }
       }
     }
   }
+
+  if (ksz >= 2 && !cl_waited) cluster_wait();
 
   if (a.append) {
     if (tid == 0) last_flag = ticket == (int)gridDim.x - 1;

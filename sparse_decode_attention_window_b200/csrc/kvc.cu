@@ -19,6 +19,7 @@
 #include "select.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "decode_tc.cuh"
 #include "profile.cuh"
 
 namespace {
@@ -121,6 +122,17 @@ bool force_simt_decode() {
   static const bool v = [] {
     const char* e = getenv("KVC_DECODE_PATH");
     return e && strcmp(e, "simt") == 0;
+  }();
+  return v;
+}
+
+// KVC_DECODE_PATH=tc routes bf16, d = 128 decode to the tcgen05 kernel (decode_tc.cuh,
+// a cross-check and measurement path: on B200 it is slower than the mma.sync kernel, see
+// that file's header); read once.
+bool force_tc_decode() {
+  static const bool v = [] {
+    const char* e = getenv("KVC_DECODE_PATH");
+    return e && strcmp(e, "tc") == 0;
   }();
   return v;
 }
@@ -287,6 +299,91 @@ kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStr
   return check_launch("kvc_decode_attn");
 }
 
+// bf16, d = 128: decode on tcgen05 (decode_tc.cuh), same work split as above; three
+// pipeline stages when they fit in shared memory, else two. Returns KVC_ERR_UNSUPPORTED
+// (without launching) when not even two fit, and the caller takes the mma.sync kernel.
+kvc_status launch_decode_tc(const kvc::DecodeParams& p, int G, int sms, cudaStream_t st, bool allow_cluster) {
+  using namespace kvc;
+  DevInfo* di = nullptr;
+  if (dev_info(&di) != KVC_OK) return KVC_ERR_CUDA;
+  int k = p.S > 0 ? sms / p.S : 0;
+  if (k > DM_MAX_CLUSTER) k = DM_MAX_CLUSTER;
+  if (!allow_cluster || force_token_split()) k = 1;
+  auto total = [&](int grid, int ksz, int nst) { return DtLayout::make(p.S, G, grid, ksz, nst).total; };
+  // the largest layout any launch below can take (grid <= SMs, records of up to 8 CTAs)
+  const size_t smem_max2 = total(sms, DM_MAX_CLUSTER, 2);
+  const size_t optin = (size_t)di->smem_optin - 2048;   // room for the kernel's static shared memory
+  if (smem_max2 > optin) return KVC_ERR_UNSUPPORTED;
+  int grid = sms;
+  for (; k >= 2; k /= 2) {
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, int> known;   // (k, device) -> resident clusters
+    int dev = 0, n = 0;
+    cudaGetDevice(&dev);
+    {
+      std::lock_guard<std::mutex> lk(mu);
+      auto it = known.find({k, dev});
+      if (it != known.end()) {
+        n = it->second;
+      } else {
+        if (set_smem(decode_tc_kernel, smem_max2, "cluster check") == KVC_OK) {
+          cudaLaunchConfig_t cfg = {};
+          cfg.gridDim = dim3((sms / k) * k);
+          cfg.blockDim = dim3(DtCfg::THREADS);
+          cfg.dynamicSmemBytes = smem_max2;
+          cudaLaunchAttribute attr[1];
+          attr[0].id = cudaLaunchAttributeClusterDimension;
+          attr[0].val.clusterDim.x = k;
+          attr[0].val.clusterDim.y = 1;
+          attr[0].val.clusterDim.z = 1;
+          cfg.attrs = attr;
+          cfg.numAttrs = 1;
+          if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel, &cfg) != cudaSuccess) n = 0;
+          cudaGetLastError();
+        }
+        known[{k, dev}] = n;
+      }
+    }
+    n = std::min(sms / k, n);
+    const long long g = (long long)n * k, sk = (long long)p.S * k;
+    if (n >= 1 && sk <= g && 4 * sk >= 3 * g) {
+      grid = (int)g;
+      break;
+    }
+  }
+  const bool cluster = k >= 2;
+  const int ksz = cluster ? k : 1;
+  const int nst = total(grid, ksz, 3) <= optin ? 3 : 2;
+  const size_t smem = total(grid, ksz, nst);
+  encode_tiled_fn enc = get_encode_tiled();
+  CUtensorMap mk, mk16, mv, mv16, mq;
+  const long long rows = p.kp_rows > 0 ? p.kp_rows : 1;
+  if (!enc || !make_map_2d_rows(&mk, enc, p.kp, 128, rows, 128) || !make_map_2d_rows(&mk16, enc, p.kp, 128, rows, 16) ||
+      !make_map_2d_rows(&mv, enc, p.vp, 128, rows, 128) || !make_map_2d_rows(&mv16, enc, p.vp, 128, rows, 16) ||
+      !make_map_2d_rows(&mq, enc, p.q, 128, (long long)p.S * G, 16))
+    return fail(KVC_ERR_CUDA, "kvc_decode_attn: cuTensorMapEncodeTiled failed");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(DtCfg::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = ksz;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cluster ? 2 : 1;
+  kvc_status rc = set_smem(decode_tc_kernel, std::max(smem, smem_max2), "kvc_decode_attn");
+  if (rc != KVC_OK) return rc;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel, mk, mk16, mv, mv16, mq, p, G, ksz, nst);
+  if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "kvc_decode_attn: launch: %s", cudaGetErrorString(e));
+  count_launches(1);
+  return check_launch("kvc_decode_attn");
+}
+
 template <typename T, int D>
 kvc_status decode_by_g(int G, const kvc::DecodeParams& p, int sms, cudaStream_t st) {
   switch (G) {
@@ -302,6 +399,10 @@ kvc_status decode_by_g(int G, const kvc::DecodeParams& p, int sms, cudaStream_t 
 kvc_status launch_decode_any(const kvc_shape* shape, const kvc::DecodeParams& p, int sms, cudaStream_t stream,
                              bool allow_cluster = true) {
   if (shape->dtype == KVC_BF16 && shape->G <= 8 && !force_simt_decode()) {
+    if (shape->d == 128 && force_tc_decode()) {
+      const kvc_status rc = launch_decode_tc(p, shape->G, sms, stream, allow_cluster);
+      if (rc != KVC_ERR_UNSUPPORTED) return rc;
+    }
     const bool pack = shape->G <= 4;   // heads and the bf16 remainder share one MMA
     if (shape->d == 128)
       return pack ? launch_decode_mma<128, true>(p, shape->G, sms, stream, allow_cluster)

@@ -376,6 +376,21 @@ def test_token_split_decode_on_few_slot_workloads():
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
+def test_tcgen05_decode_path_on_bf16_workloads():
+    """The tcgen05 decode (opt-in cross-check path, d = 128) passes the same oracle checks,
+    including full-size llama8b and the fused-append overflow case."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, KVC_DECODE_PATH="tc")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        "-k", "llama8b_shape_small_context or zigzag_small or chunk_small or fastgen_small "
+                              "or llama8b_full_size or separate_append or fused_append_decode_overflow "
+                              "or ragged_context_lengths or gqa_group_sizes"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
 # ---------------------------------------------------------------- next rows
 def test_retained_mass_matches_oracle():
     """Attention retained by the selection (ZigZagKV's attention loss is 0.9 minus it)."""
