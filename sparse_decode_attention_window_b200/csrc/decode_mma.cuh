@@ -33,7 +33,8 @@ struct DmCfg {
   static constexpr int REGION = TILE * 128;          // one k-block of one tile (8 KB)
   static constexpr int STAGE_BYTES = 2 * KB * REGION;
   static constexpr int STAGES = 4;
-  static constexpr int CONS_WARPS = 4;               // each consumes one 16-token m-tile per stage
+  static constexpr int GROUP_WARPS = 4;              // a group takes a tile: one 16-token m-tile per warp
+  static constexpr int CONS_WARPS = 2 * GROUP_WARPS; // two groups take alternate tiles
   static constexpr int CONS_THREADS = CONS_WARPS * 32;
   static constexpr int THREADS = CONS_THREADS + 32;
   static constexpr int KSTEPS = D / 16;
@@ -278,7 +279,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     abort_flag = 0;
     for (int i = 0; i < C::STAGES; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], C::CONS_WARPS);
+      mbar_init(&empty[i], C::GROUP_WARPS);
     }
     mbar_init(rec_bar, 1);
     fence_mbar_init();
@@ -407,7 +408,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
           const int row0 = (int)(offs[s] + (u - P[s]));
           unsigned char* kdst = stages + stage * C::STAGE_BYTES;
           unsigned char* vdst = kdst + C::KB * C::REGION;
-          const uint32_t qb = u == t ? q_bytes : 0u;
+          const uint32_t qb = q_bytes;   // q rides with every tile: either group may start the segment
           if (rows == C::TILE) {
             mbar_arrive_expect_tx(&full[stage], 2 * C::KB * C::REGION + qb);
 #pragma unroll
@@ -440,10 +441,13 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     }
     __syncwarp();
   } else if (active || in_slot_cluster) {
-    // ---------------- consumers: warp cw owns rows [16 cw, 16 cw + 16) of every tile
+    // ---------------- consumers: group cw / 4 takes the tiles of its parity (counted over the
+    // CTA), and warp cw owns rows [16 (cw % 4), + 16) of each of them; two groups keep two
+    // tiles' dependency chains in flight on every SM sub-partition
     const int cw = warp;
+    const int grp = cw / C::GROUP_WARPS;
     const int g = lane >> 2, qd = lane & 3;                 // fragment row group, column pair
-    const int mrow0 = 16 * cw;
+    const int mrow0 = 16 * (cw % C::GROUP_WARPS);
     const int lm_j = lane >> 3, lm_r = lane & 7;            // ldmatrix lane roles
     // heads of this thread's S^T / O^T columns 2qd and 2qd + 1
     const int hc0 = PACK ? 2 * (qd & 1) : 2 * qd, hc1 = hc0 + 1;
@@ -453,6 +457,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     const int qhead = PACK ? (g & 3) : g;                   // head of Q^T column g
     int stage = 0;
     uint32_t ph = 0;
+    long long tile_k = 0;                                   // tiles of this CTA so far
     bool aborted = false;
     bool pending_empty = in_slot_cluster && !active;       // a cluster CTA without tokens: one empty record
     for (long long t = b0; (t < b1 && !aborted) || pending_empty;) {
@@ -466,14 +471,20 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
 #pragma unroll
       for (int dt = 0; dt < C::DTILES; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
 
-      for (long long u = t; u < seg_end; u += C::TILE) {
+      bool have_q = false;
+      for (long long u = t; u < seg_end; u += C::TILE, ++tile_k) {
+        if ((int)(tile_k & 1) != grp) {      // the other group's tile
+          if (++stage == C::STAGES) { stage = 0; ph ^= 1; }
+          continue;
+        }
         const int rows = (int)min((long long)C::TILE, seg_end - u);
-        if (!mbar_wait(&full[stage], ph)) {   // every consumer warp waits on this barrier: all stop here
+        if (!mbar_wait(&full[stage], ph)) {   // the group's warps wait on this barrier: all stop here
           *(volatile int*)&abort_flag = 1;
           aborted = true;
           break;
         }
-        if (u == t) {
+        if (!have_q) {
+          have_q = true;
           // Q^T operand (k = d, n = head) from the copy that came with this tile
           const unsigned char* qs = qbuf + (size_t)stage * q_bytes;
 #pragma unroll
@@ -611,7 +622,12 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         if (lane == 0) mbar_arrive(&empty[stage]);
         if (++stage == C::STAGES) { stage = 0; ph ^= 1; }
       }
-      if (aborted) break;
+      // the two groups wait on different barriers: agree on an abort before any barrier
+      // that needs both of them
+      if (named_bar_or(1, C::CONS_THREADS, aborted)) {
+        aborted = true;
+        break;
+      }
 
       // ---- the warp's totals: l over its 8 row groups; PACK adds the remainder columns
 #pragma unroll
