@@ -32,7 +32,7 @@ struct DmCfg {
   static constexpr int TILE = 64;                    // tokens per stage
   static constexpr int REGION = TILE * 128;          // one k-block of one tile (8 KB)
   static constexpr int STAGE_BYTES = 2 * KB * REGION;
-  static constexpr int STAGES = 4;
+  static constexpr int MAX_STAGES = 6;              // pipeline depth chosen at launch: 4 or 6 (even, see the launcher)
   static constexpr int GROUP_WARPS = 4;              // a group takes a tile: one 16-token m-tile per warp
   static constexpr int CONS_WARPS = 2 * GROUP_WARPS; // two groups take alternate tiles
   static constexpr int CONS_THREADS = CONS_WARPS * 32;
@@ -53,13 +53,13 @@ constexpr int DM_MAX_CLUSTER = 8;
 struct DmLayout {
   size_t stages, qbuf, bars, P, offs, wm, wo, xr, app, total;
   template <int D>
-  KVC_HD static DmLayout make(int S, int G, int grid) {
+  KVC_HD static DmLayout make(int S, int G, int grid, int nst) {
     using C = DmCfg<D>;
     DmLayout l{};
     size_t o = 0;
-    l.stages = o;  o += (size_t)C::STAGES * C::STAGE_BYTES;          // 1024-byte aligned base
-    l.qbuf = o;    o += (size_t)C::STAGES * G * D * 2;               // the segment's q, one per stage
-    l.bars = o;    o += (2 * C::STAGES + 1) * sizeof(uint64_t);      // full, empty, rank 0's record barrier
+    l.stages = o;  o += (size_t)nst * C::STAGE_BYTES;                // 1024-byte aligned base
+    l.qbuf = o;    o += (size_t)nst * G * D * 2;                     // the slot's q, one per stage
+    l.bars = o;    o += (2 * C::MAX_STAGES + 1) * sizeof(uint64_t);  // full, empty, rank 0's record barrier
     l.P = o;       o += (size_t)(S + 1) * sizeof(long long);
     l.offs = o;    o += (size_t)S * sizeof(long long);
     l.wm = o;      o += 2 * C::CONS_WARPS * 8 * sizeof(float);       // per-warp max and sum, 8 heads
@@ -76,8 +76,8 @@ struct DmLayout {
 };
 
 template <int D>
-inline size_t decode_mma_smem_bytes(int S, int G, int grid) {
-  return DmLayout::make<D>(S, G, grid).total;
+inline size_t decode_mma_smem_bytes(int S, int G, int grid, int nst) {
+  return DmLayout::make<D>(S, G, grid, nst).total;
 }
 
 KVC_DEV void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -248,18 +248,18 @@ template <int D, bool PACK>
 __global__ void __launch_bounds__(DmCfg<D>::THREADS, 1)
 decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constant__ CUtensorMap mk16,
                   const __grid_constant__ CUtensorMap mv64, const __grid_constant__ CUtensorMap mv16,
-                  DecodeParams a, int G, int ksz) {
+                  DecodeParams a, int G, int ksz, int nst) {
   using C = DmCfg<D>;
   extern __shared__ __align__(1024) unsigned char dm_raw[];
   const uint32_t raw = smem_u32(dm_raw);
   unsigned char* sm = dm_raw + (((raw + 1023u) & ~1023u) - raw);
   const int S = a.S;
-  const DmLayout lay = DmLayout::make<D>(S, G, gridDim.x);
+  const DmLayout lay = DmLayout::make<D>(S, G, gridDim.x, nst);
   unsigned char* stages = sm + lay.stages;
   unsigned char* qbuf = sm + lay.qbuf;
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + lay.bars);
-  uint64_t* empty = full + C::STAGES;
-  uint64_t* rec_bar = empty + C::STAGES;   // rank 0 of a slot cluster: the other CTAs' records (st.async bytes)
+  uint64_t* empty = full + C::MAX_STAGES;
+  uint64_t* rec_bar = empty + C::MAX_STAGES;   // rank 0 of a slot cluster: the other CTAs' records (st.async bytes)
   long long* P = reinterpret_cast<long long*>(sm + lay.P);
   long long* offs = reinterpret_cast<long long*>(sm + lay.offs);
   float* wm = reinterpret_cast<float*>(sm + lay.wm);        // [warp][8] maxima
@@ -277,7 +277,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   if (tid == 0) {
     max_len_sh = 0;
     abort_flag = 0;
-    for (int i = 0; i < C::STAGES; ++i) {
+    for (int i = 0; i < nst; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], C::GROUP_WARPS);
     }
@@ -400,8 +400,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         const long long seg_end = min(b1, P[s + 1]);
         for (long long u = t; u < seg_end; u += C::TILE) {
           const int rows = (int)min((long long)C::TILE, seg_end - u);
-          // the first STAGES tiles find their stages free
-          if ((issued >= C::STAGES && !mbar_wait(&empty[stage], ph ^ 1)) || *(volatile int*)&abort_flag) {
+          // the first nst tiles find their stages free
+          if ((issued >= nst && !mbar_wait(&empty[stage], ph ^ 1)) || *(volatile int*)&abort_flag) {
             ok = false;
             break;
           }
@@ -430,14 +430,14 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
             bulk_g2s(qbuf + (size_t)stage * q_bytes, static_cast<const unsigned char*>(a.q) + (size_t)s * q_bytes,
                      q_bytes, &full[stage]);
           ++issued;
-          if (++stage == C::STAGES) { stage = 0; ph ^= 1; }
+          if (++stage == nst) { stage = 0; ph ^= 1; }
         }
         t = seg_end;
       }
       if (!ok) *(volatile int*)&abort_flag = 1;
       // every load issued has landed before the CTA may exit
-      for (long long k = issued > C::STAGES ? issued - C::STAGES : 0; k < issued; ++k)
-        mbar_wait(&full[k % C::STAGES], (uint32_t)((k / C::STAGES) & 1));
+      for (long long k = issued > nst ? issued - nst : 0; k < issued; ++k)
+        mbar_wait(&full[k % nst], (uint32_t)((k / nst) & 1));
     }
     __syncwarp();
   } else if (active || in_slot_cluster) {
@@ -474,7 +474,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       bool have_q = false;
       for (long long u = t; u < seg_end; u += C::TILE, ++tile_k) {
         if ((int)(tile_k & 1) != grp) {      // the other group's tile
-          if (++stage == C::STAGES) { stage = 0; ph ^= 1; }
+          if (++stage == nst) { stage = 0; ph ^= 1; }
           continue;
         }
         const int rows = (int)min((long long)C::TILE, seg_end - u);
@@ -620,7 +620,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         if (patched) fence_proxy_async();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[stage]);
-        if (++stage == C::STAGES) { stage = 0; ph ^= 1; }
+        if (++stage == nst) { stage = 0; ph ^= 1; }
       }
       // the two groups wait on different barriers: agree on an abort before any barrier
       // that needs both of them

@@ -297,6 +297,50 @@ def test_decode_is_independent_of_how_tokens_split_over_ctas():
         P.check_out(_np(out[s * G:(s + 1) * G]), ref, "bf16", f"slot {s} vs oracle")
 
 
+@pytest.mark.parametrize("G,S,fused", [(4, 4096, True), (8, 2500, False), (2, 4096, False)])
+def test_maximum_slot_counts(G, S, fused):
+    """Large slot counts (up to the 4096 the decode takes): short ragged lengths including
+    empty slots, sampled slots against the oracle."""
+    import sparse_decode_attention_window_b200 as kvc
+    d = 128
+    g = torch.Generator().manual_seed(S + G)
+    lens = torch.randint(0, 40, (S,), generator=g, dtype=torch.int32)
+    sh = kvc.make_shape(S, G, d, 64, 0, S, 1, torch.bfloat16)
+    count = lens.cuda()
+    off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    cap = torch.empty(S, dtype=torch.int32, device="cuda")
+    kvc.kvc_layout(count, 1, off, cap)
+    rows = int(off[-1])
+    kp = torch.randn(rows, d, generator=g).to(torch.bfloat16).cuda()
+    vp = torch.randn(rows, d, generator=g).to(torch.bfloat16).cuda()
+    q = torch.randn(S * G, d, generator=g).to(torch.bfloat16).cuda()
+    kn = torch.randn(S, d, generator=g).to(torch.bfloat16).cuda()
+    vn = torch.randn(S, d, generator=g).to(torch.bfloat16).cuda()
+    out = torch.empty((S * G, d), device="cuda")
+    ws = torch.zeros(kvc.kvc_workspace_size(kvc.KVC_WS_DECODE, sh), dtype=torch.uint8, device="cuda")
+    ln = count.clone()
+    if fused:
+        kvc.kvc_append_decode(sh, kn, vn, q, kp, vp, off, cap, ln, out, ws)
+    else:
+        kvc.kvc_decode_attn(sh, q, kp, vp, off, ln, out, ws)
+    kvc.kvc_get_status()
+    o = _np(out)
+    offs = _np(off)
+    for s in list(range(0, S, 97)) + [S - 1]:
+        n = int(lens[s])
+        keys, vals = kp[offs[s]:offs[s] + n].cpu(), vp[offs[s]:offs[s] + n].cpu()
+        if fused:
+            keys, vals = torch.cat([keys, kn[s:s + 1].cpu()]), torch.cat([vals, vn[s:s + 1].cpu()])
+            n += 1
+        if n == 0:
+            assert (o[s * G:(s + 1) * G] == 0).all()
+            continue
+        ref = O.decode_attention(q[s * G:(s + 1) * G].cpu(), keys, vals, [0, n], [n], G)
+        P.check_out(o[s * G:(s + 1) * G], ref, "bf16", f"slot {s}")
+    if fused:
+        assert (_np(ln) == _np(count) + 1).all()
+
+
 def test_wide_window_takes_cuda_core_scoring_path():
     """G*w = 256 rows exceeds the tensor-core tile: scoring runs on the CUDA-core kernels;
     decode with G = 8 query heads per KV head."""
