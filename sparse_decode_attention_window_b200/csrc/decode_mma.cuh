@@ -47,6 +47,7 @@ struct DmCfg {
 // rescale; probabilities then stay below 2^8, far inside fp32 and the bf16 hi/lo split.
 constexpr float DM_LAZY_LOG2 = 8.f;
 constexpr int DM_MIN_TOKENS_PER_CTA = 64;            // token split: no CTA gets less than a tile
+constexpr long long DM_SEG_COST = 128;               // token split: fixed work of one slot segment, in tokens
 constexpr int DM_MAX_CLUSTER = 8;
 
 // Shared-memory layout of decode_mma_kernel (host and device agree on it).
@@ -64,11 +65,9 @@ struct DmLayout {
     l.offs = o;    o += (size_t)S * sizeof(long long);
     l.wm = o;      o += 2 * C::CONS_WARPS * 8 * sizeof(float);       // per-warp max and sum, 8 heads
     l.wo = o;      o += (size_t)C::CONS_WARPS * G * C::WO_STRIDE * sizeof(float);
-    // token split: scale table of the merge [grid][G] + 1/sum [8]; per-slot clusters:
-    // the k CTA records [k][G*D + 2G] that rank 0 merges
-    const size_t tok = ((size_t)grid * G + 8) * sizeof(float);
+    // per-slot clusters: the k CTA records [k][G*D + 2G, padded] that rank 0 merges
     const size_t clu = 2 * S <= grid ? (size_t)DM_MAX_CLUSTER * partial_stride(G, D) * sizeof(float) : 0;
-    l.xr = o;      o += (tok > clu ? tok : clu);
+    l.xr = o;      o += clu;
     l.app = o;     o += (size_t)S;
     l.total = o + 1024 + 16;                                          // base alignment slack
     return l;
@@ -182,49 +181,46 @@ KVC_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
 }
 
 // The last CTA to finish slot s in the token split merges the slot's CTA partials
-// (CTAs cfirst..clast, stored consecutively at index c + s): warp w finds the maximum
-// and the scaled sum of heads w, w + 4, ... over all partials (lanes stride the
-// partials), then each thread folds float4 columns of the outputs over the partials
-// with independent loads. Runs on the CTA's consumer threads.
-KVC_DEV void merge_partials_par(const DecodeParams& a, int s, int G, int D, int cfirst, int clast, float* sc_tab,
-                                int tid, int nthr) {
+// (CTAs cfirst..clast, stored consecutively at index c + s). Each thread owns one float4
+// column of the outputs and folds the partials in groups of 8 whose (max, sum, column)
+// loads are issued together, so up to 8 partials cost one round trip to L2.
+KVC_DEV void merge_partials_par(const DecodeParams& a, int s, int G, int D, int cfirst, int clast, int tid,
+                                int nthr) {
   const int np = clast - cfirst + 1;
   const size_t stride = (size_t)partial_stride(G, D);
   const float* base = a.partial + (size_t)(cfirst + s) * stride;
-  float* linv = sc_tab + (size_t)np * G;   // [8]
-  const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
-  for (int h = warp; h < G; h += nw) {
-    float M = -INFINITY;
-    for (int p = lane; p < np; p += 32) M = fmaxf(M, __ldcg(base + (size_t)p * stride + (size_t)G * D + h));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float Lt = 0.f;
-    for (int p = lane; p < np; p += 32) {
-      const float m = __ldcg(base + (size_t)p * stride + (size_t)G * D + h);
-      const float l = __ldcg(base + (size_t)p * stride + (size_t)G * D + G + h);
-      const float sc = m == -INFINITY ? 0.f : ex2_ftz(m - M);
-      sc_tab[p * G + h] = sc;
-      Lt += l * sc;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) Lt += __shfl_xor_sync(0xffffffffu, Lt, o);
-    if (lane == 0) linv[h] = Lt > 0.f ? 1.f / Lt : 0.f;
-  }
-  named_bar_sync(1, nthr);
   const int nq = G * D / 4;
   for (int c4 = tid; c4 < nq; c4 += nthr) {
     const int h = (c4 * 4) / D;
+    float M = -INFINITY, Lt = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int p = 0; p < np; ++p) {
-      const float sc = sc_tab[p * G + h];
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(base + (size_t)p * stride) + c4);
-      acc.x += sc * v.x;
-      acc.y += sc * v.y;
-      acc.z += sc * v.z;
-      acc.w += sc * v.w;
+    for (int p0 = 0; p0 < np; p0 += 8) {
+      float m[8], l[8];
+      float4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const bool in = p0 + k < np;
+        const float* pp = base + (size_t)(p0 + k) * stride;
+        m[k] = in ? __ldcg(pp + (size_t)G * D + h) : -INFINITY;
+        l[k] = in ? __ldcg(pp + (size_t)G * D + G + h) : 0.f;
+        v[k] = in ? __ldcg(reinterpret_cast<const float4*>(pp) + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float Mn = M;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) Mn = fmaxf(Mn, m[k]);
+      if (Mn == -INFINITY) continue;
+      const float sc = M == -INFINITY ? 0.f : ex2_ftz(M - Mn);
+      Lt *= sc;
+      acc.x *= sc; acc.y *= sc; acc.z *= sc; acc.w *= sc;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float w = m[k] == -INFINITY ? 0.f : ex2_ftz(m[k] - Mn);
+        Lt += l[k] * w;
+        acc.x += v[k].x * w; acc.y += v[k].y * w; acc.z += v[k].z * w; acc.w += v[k].w * w;
+      }
+      M = Mn;
     }
-    const float li = linv[h];
+    const float li = Lt > 0.f ? 1.f / Lt : 0.f;
     reinterpret_cast<float4*>(a.out + (size_t)s * G * D)[c4] = make_float4(acc.x * li, acc.y * li, acc.z * li, acc.w * li);
   }
 }
@@ -351,6 +347,20 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
 
   const long long N = P[S];
   const int nC = gridDim.x, c = blockIdx.x;
+  // Token split by cost: every slot segment a CTA touches costs DM_SEG_COST tokens' worth
+  // of fixed work (its last partial tile, the combine, the output or partial), so token t
+  // of slot s sits at cost t + (s + 1) DM_SEG_COST and CTAs get equal cost ranges; a CTA
+  // that crosses many short slots gets fewer tokens.
+  const long long T = N + (long long)S * DM_SEG_COST;
+  auto token_at_cost = [&](long long x) -> long long {   // first token whose cost is >= x
+    if (x >= T) return N;
+    int lo = 0, hi = S - 1;                                // last slot whose cost range starts <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (P[mid] + (long long)mid * DM_SEG_COST <= x) lo = mid; else hi = mid - 1;
+    }
+    return max(P[lo], x - (long long)(lo + 1) * DM_SEG_COST);
+  };
   // per-slot clusters: launched in clusters, every slot has one, they fill >= 3/4 of
   // the grid, and the lengths are near uniform (the same test in every CTA)
   const bool per_slot = ksz >= 2 && (long long)S * ksz <= nC && 4LL * S * ksz >= 3LL * nC &&
@@ -365,9 +375,11 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       if (P[s + 1] == P[s])
         for (int e = tid; e < G * D; e += blockDim.x) a.out[(size_t)s * G * D + e] = 0.f;
     nE = (int)min((long long)nC, (N + DM_MIN_TOKENS_PER_CTA - 1) / DM_MIN_TOKENS_PER_CTA);
-    active = N > 0 && c < nE;
-    b0 = active ? (long long)c * N / nE : 0;
-    b1 = active ? (long long)(c + 1) * N / nE : 0;
+    if (N > 0 && c < nE) {
+      b0 = token_at_cost((long long)c * T / nE);
+      b1 = token_at_cost((long long)(c + 1) * T / nE);
+    }
+    active = b1 > b0;
   } else if (in_slot_cluster) {
     const long long r = (long long)cluster_rank(), ns = P[my_cluster + 1] - P[my_cluster];
     b0 = P[my_cluster] + r * ns / ksz;
@@ -384,7 +396,11 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     }
     return lo;
   };
-  auto cta_of = [&](long long t) { return (int)(((t + 1) * nE - 1) / N); };
+  // the CTA whose cost range holds token t of slot s
+  auto cta_of = [&](long long t, int s) {
+    const long long x = t + (long long)(s + 1) * DM_SEG_COST;
+    return (int)(((x + 1) * nE - 1) / T);
+  };
   const uint32_t q_bytes = (uint32_t)(G * D * 2);
 
   if (warp == C::CONS_WARPS) {
@@ -674,7 +690,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       }
       named_bar_sync(1, C::CONS_THREADS);
 
-      const int cfirst = per_slot ? 0 : cta_of(P[s]), clast = per_slot ? 0 : cta_of(P[s + 1] - 1);
+      const int cfirst = per_slot ? 0 : cta_of(P[s], s), clast = per_slot ? 0 : cta_of(P[s + 1] - 1, s);
       const bool single = !per_slot && cfirst == clast;
       float* mypart = a.partial + (size_t)(c + s) * partial_stride(G, D);
       const uint32_t my_rank = per_slot ? cluster_rank() : 0u;
@@ -728,7 +744,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         if (tid == 0) last_flag = slot_ticket(&a.counters[s], clast - cfirst);
         named_bar_sync(1, C::CONS_THREADS);
         if (last_flag) {
-          merge_partials_par(a, s, G, D, cfirst, clast, xr, tid, C::CONS_THREADS);
+          merge_partials_par(a, s, G, D, cfirst, clast, tid, C::CONS_THREADS);
           if (tid == 0) a.counters[s] = 0;
         }
       }

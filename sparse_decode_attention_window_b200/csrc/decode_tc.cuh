@@ -75,12 +75,10 @@ struct DtLayout {
     l.P = o;      o += (size_t)(S + 1) * sizeof(long long);
     l.offs = o;   o += (size_t)S * sizeof(long long);
     l.red = o;    o += 6 * C::CONS_WARPS * 8 * sizeof(float);     // maxima, sums [warp][8]; merge weights [8][8], 1/sum [8]
-    // token split: the merge's scale table [grid][G] + 1/sum [8]; per-slot clusters: the
-    // ksz records that rank 0 merges, 16-byte aligned
-    const size_t tok = ((size_t)grid * G + 8) * sizeof(float);
+    // per-slot clusters: the ksz records that rank 0 merges, 16-byte aligned
     const size_t clu = ksz >= 2 ? (size_t)ksz * partial_stride(G, C::D) * sizeof(float) : 0;
     o = (o + 15) & ~(size_t)15;
-    l.xr = o;     o += (tok > clu ? tok : clu);
+    l.xr = o;     o += clu;
     l.app = o;    o += (size_t)S;
     l.total = o + 1024 + 16;                                // base alignment slack
     return l;
@@ -621,7 +619,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mk, const __grid_constant__
           if (tid == 0) last_flag = slot_ticket(&a.counters[s], clast - cfirst);
           named_bar_sync(2, C::CONS_THREADS);
           if (last_flag) {
-            merge_partials_par(a, s, G, D, cfirst, clast, xr, tid, C::CONS_THREADS);
+            merge_partials_par(a, s, G, D, cfirst, clast, tid, C::CONS_THREADS);
             if (tid == 0) a.counters[s] = 0;
           }
         }
