@@ -145,6 +145,64 @@ KVC_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// ---------------------------------------------------------------- thread-block clusters
+KVC_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+
+// Map a local shared-memory address to the same offset in CTA `rank` of the cluster.
+KVC_DEV uint32_t map_to_rank(const void* local, uint32_t rank) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+  return ra;
+}
+// Asynchronous 4-byte store into another CTA's shared memory; its completion counts 4
+// bytes on that CTA's mbarrier.
+KVC_DEV void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+KVC_DEV void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
+KVC_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// Bounded wait with cluster-scope acquire (data that other CTAs sent with st.async).
+KVC_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  auto try_once = [&]() {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+  };
+  if (try_once()) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (try_once()) return true;
+    if (global_timer_ns() - t0 > KVC_WAIT_LIMIT_NS) {
+      kvc_flag(KVC_DEVERR_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Asynchronous 8-byte store into another CTA's shared memory; its completion counts 8
+// bytes on that CTA's mbarrier.
+KVC_DEV void st_async_f32x2(uint32_t remote_addr, float x, float y, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];" ::"r"(remote_addr),
+               "r"(__float_as_uint(x)), "r"(__float_as_uint(y)), "r"(remote_bar)
+               : "memory");
+}
+
 // Plain (untiled) bulk copy global -> shared, completion counted on `bar`.
 // Both addresses 16-byte aligned, bytes a multiple of 16.
 KVC_DEV void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {

@@ -108,55 +108,6 @@ KVC_DEV uint32_t pack_bf16(float lo, float hi) {
 }
 KVC_DEV float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
-KVC_DEV uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-
-// Map a local shared-memory address to the same offset in CTA `rank` of the cluster.
-KVC_DEV uint32_t map_to_rank(const void* local, uint32_t rank) {
-  uint32_t ra;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
-  return ra;
-}
-// Asynchronous 4-byte store into another CTA's shared memory; its completion counts 4
-// bytes on that CTA's mbarrier.
-KVC_DEV void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
-               "r"(__float_as_uint(v)), "r"(remote_bar)
-               : "memory");
-}
-KVC_DEV void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
-KVC_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
-
-// Bounded wait with cluster-scope acquire (data that other CTAs sent with st.async).
-KVC_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
-  auto try_once = [&]() {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-  };
-  if (try_once()) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (try_once()) return true;
-    if (global_timer_ns() - t0 > KVC_WAIT_LIMIT_NS) {
-      kvc_flag(KVC_DEVERR_WAIT_TIMEOUT);
-      return false;
-    }
-  }
-}
-
 // Byte offset of (row, 16-byte chunk) in a 128-byte-swizzled region of 128-byte rows.
 KVC_DEV uint32_t swz(int row, int chunk) { return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4)); }
 

@@ -117,6 +117,16 @@ bool force_simt() {
   return v;
 }
 
+// KVC_SCORE_PATH=twopass keeps tensor-core scoring in its two-launch form (pass 1, merge,
+// pass 2) where the fused slot-cluster kernel would run (cross-checks); read once.
+bool force_two_pass_score() {
+  static const bool v = [] {
+    const char* e = getenv("KVC_SCORE_PATH");
+    return e && strcmp(e, "twopass") == 0;
+  }();
+  return v;
+}
+
 // KVC_DECODE_PATH=simt routes bf16 decode to the CUDA-core kernel (cross-checks); read once.
 bool force_simt_decode() {
   static const bool v = [] {
@@ -531,7 +541,7 @@ kvc_status kvc_score(const kvc_shape* shape, const void* q_win, const void* k, c
   if (kvc::tc_supported(shape, di->cc_major, di->cc_minor) && !force_simt()) {
     unsigned nl = 0;
     rc = kvc::tc_score(shape, q_win, k, chunk_end, C, row_lse, score, part, lse, wsb + w.keys_off, di->sms, stream,
-                       &fail, &nl);
+                       &fail, &nl, force_two_pass_score());
     count_launches(nl);
     if (rc != KVC_OK) return rc;
     return check_launch("kvc_score");

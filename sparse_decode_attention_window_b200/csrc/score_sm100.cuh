@@ -24,6 +24,8 @@
 // Chunk keys are first gathered into a contiguous buffer (one row per chunk).
 #pragma once
 #include <algorithm>
+#include <map>
+#include <mutex>
 #include "common.cuh"
 #include "cache.cuh"
 
@@ -37,6 +39,7 @@ constexpr int TC_STAGES = 4;
 constexpr int TC_EPI_WARPS = 8;   // two per SM sub-partition; warp pair (w, w+4) splits the 128 columns
 constexpr int TC_THREADS = 32 * (2 + TC_EPI_WARPS);
 constexpr int TC_TMEM_COLS = 256; // two 128-column fp32 accumulators
+constexpr int TC_MAX_CLUSTER = 16; // fused mode: CTAs per slot (16 needs the non-portable cluster size)
 
 // ---------------------------------------------------------------- PTX wrappers (tcgen05)
 KVC_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -128,7 +131,9 @@ struct TcSmem {
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;     // tmem addr, flags
   static constexpr int LSE_OFF = MISC_OFF + 64;           // pass 2: lse2[128], win index [128]
   static constexpr int XCH_OFF = LSE_OFF + 2 * TC_ROWS * 4; // half-to-half exchange [128] float2
-  static constexpr int TOTAL = XCH_OFF + TC_ROWS * 8;
+  static constexpr int XALL_OFF = XCH_OFF + TC_ROWS * 8;    // fused mode: row stats of every CTA [16][128] float2
+  static constexpr int XBAR_OFF = XALL_OFF + TC_MAX_CLUSTER * TC_ROWS * 8;
+  static constexpr int TOTAL = XBAR_OFF + 8;
   static constexpr int ALLOC = TOTAL + 1024;              // room to align the base to 1024 B
 };
 
@@ -136,7 +141,7 @@ struct TcParams {
   int S, N, L, w, R, G;
   int tiles;          // tiles per slot = ceil(N / 128)
   int tpi;            // tiles per work item
-  int nsplit;         // work items per slot = ceil(tiles / tpi)
+  int nsplit;         // work items per slot = ceil(tiles / tpi) (fused mode: the cluster size)
   float scale2;       // log2(e) / sqrt(d)
   const int32_t* key_pos;  // chunk mode: position of key n (chunk_end); NULL: key n at position n
   float2* part;       // pass 1 out: [S][nsplit][R] (max2, sum)
@@ -155,7 +160,12 @@ KVC_DEV int visible_keys(const TcParams& p, int rowpos) {
   return lo;
 }
 
-// PASS = 1: row statistics; PASS = 2: column sums.
+// PASS = 1: row statistics; PASS = 2: column sums; PASS = 3: both, fused - launched in
+// clusters of nsplit CTAs, cluster j scores slot j, CTA r its r-th key range: pass 1 over
+// the range, every CTA sends its rows' (max, sum) to every CTA of the cluster (st.async,
+// counted on an mbarrier in the receiver, so the TMA and MMA warps never wait on the
+// exchange), each CTA folds them into the rows' normalisers, and pass 2 re-reads the same
+// key tiles while they are still in L2.
 template <int D, int PASS>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k, TcParams p) {
@@ -178,6 +188,9 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
   float* lse_s = reinterpret_cast<float*>(sm + L_::LSE_OFF);
   int* win_s = reinterpret_cast<int*>(sm + L_::LSE_OFF + TC_ROWS * 4);
   float2* xch = reinterpret_cast<float2*>(sm + L_::XCH_OFF);
+  float2* xall = reinterpret_cast<float2*>(sm + L_::XALL_OFF);   // fused: [rank][row] (max2, sum)
+  uint64_t* xbar = reinterpret_cast<uint64_t*>(sm + L_::XBAR_OFF);
+  constexpr int NPASS = PASS == 3 ? 2 : 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.S * p.nsplit;
@@ -190,6 +203,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
+    mbar_init(xbar, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tm_full[b], 1);
       mbar_init(&tm_empty[b], TC_EPI_WARPS / 2);
@@ -202,6 +216,10 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     prefetch_tensormap(&map_k);
   }
   if (warp == 1) tc_alloc(tmem_slot, TC_TMEM_COLS);
+  // fused: every CTA's barriers are initialised before any CTA of the cluster sends to it
+  // (the matching wait precedes the first st.async, or ends the kernel)
+  if (PASS == 3) cluster_arrive_relaxed();
+  bool cl_waited = false;
   if (threadIdx.x < TC_ROWS) {
     // window index of pass-2 column r (rows beyond R never match)
     win_s[threadIdx.x] = threadIdx.x < p.R ? threadIdx.x % p.w : 0x40000000;
@@ -227,7 +245,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         for (int kb = 0; kb < L_::KB; ++kb) tma_load_3d(q_s + kb * TC_ROWS * 128, &map_q, kb * 64, 0, s, q_full);
         qph ^= 1;
         ++q_issued;
-        for (int j = j0; j < j1; ++j) {
+        for (int jj = j0; jj < j0 + NPASS * (j1 - j0) && ok; ++jj) {   // fused: the range twice
+          const int j = j0 + (jj - j0) % (j1 - j0);
           if (!mbar_wait(&kv_empty[st], ph ^ 1) || *abort_flag) { ok = false; break; }
           mbar_arrive_expect_tx(&kv_full[st], L_::K_BYTES);
           unsigned char* dst = k_s + st * L_::K_BYTES;
@@ -259,7 +278,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         const int j0 = sp * p.tpi, j1 = min(p.tiles, j0 + p.tpi);
         if (!mbar_wait(q_full, qph) || *abort_flag) { ok = false; break; }
         qph ^= 1;
-        for (int j = j0; j < j1; ++j) {
+        for (int jj = j0; jj < j0 + NPASS * (j1 - j0); ++jj) {   // fused: pass 1, then pass 2
+          const bool rows_on_lanes = PASS == 1 || (PASS == 3 && jj < j1);   // D = Q K^T
           if (!mbar_wait(&kv_full[st], ph) || !mbar_wait(&tm_empty[b], tph ^ 1) || *abort_flag) {
             ok = false;
             break;
@@ -273,8 +293,8 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
             for (int kk = 0; kk < 4; ++kk) {   // 4 x K=16 per 64-element k-block (+32 B each)
               const uint32_t qa = q_addr + kb * TC_ROWS * 128 + kk * 32;
               const uint32_t ka = k_addr + kb * TC_TILE * 128 + kk * 32;
-              const uint64_t a = PASS == 1 ? smem_desc_sw128(qa) : smem_desc_sw128(ka);
-              const uint64_t bb = PASS == 1 ? smem_desc_sw128(ka) : smem_desc_sw128(qa);
+              const uint64_t a = rows_on_lanes ? smem_desc_sw128(qa) : smem_desc_sw128(ka);
+              const uint64_t bb = rows_on_lanes ? smem_desc_sw128(ka) : smem_desc_sw128(qa);
               tc_mma(d_tmem, a, bb, idesc, (kb | kk) != 0);
             }
           }
@@ -311,16 +331,36 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
     uint32_t tph = 0;                             // phase of this group's accumulator barrier
     const int Lw = p.L - p.w;
     bool ok = true;
+    bool x_waited = false;                        // fused: the exchange barrier was waited on
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
       const int s = item / p.nsplit, sp = item - s * p.nsplit;
-      const int j0 = sp * p.tpi, j1 = min(p.tiles, j0 + p.tpi);
+      const int j0 = sp * p.tpi, j1 = max(j0, min(p.tiles, j0 + p.tpi));
+      for (int ps = 0; ps < NPASS && ok; ++ps) {
+      const bool p1 = PASS == 1 || (PASS == 3 && ps == 0);   // this sweep: row statistics
       float m2 = -INFINITY, lsum = 0.f;            // pass 1 running stats of row t over this group's tiles
       int vis = 0;
-      if (PASS == 1) {
+      if (p1) {
         vis = t < p.R ? visible_keys(p, Lw + (t % p.w)) : 0;
       } else {
         named_bar_sync(1, NEPI);                    // previous item's lse_s reads are done
-        if (grp == 0) lse_s[t] = t < p.R ? p.lse2[(size_t)s * p.R + t] : INFINITY;
+        if (grp == 0) {
+          if (PASS == 2) {
+            lse_s[t] = t < p.R ? p.lse2[(size_t)s * p.R + t] : INFINITY;
+          } else {
+            // fused: every CTA of the cluster sent its rows' (max2, sum); fold them
+            x_waited = true;
+            if (!mbar_wait_cluster(xbar, 0)) ok = false;
+            float M = -INFINITY;
+            for (int r = 0; r < p.nsplit; ++r) M = fmaxf(M, xall[r * TC_ROWS + t].x);
+            float l = 0.f;
+            if (M != -INFINITY)
+              for (int r = 0; r < p.nsplit; ++r) {
+                const float2 q = xall[r * TC_ROWS + t];
+                if (q.x != -INFINITY) l += q.y * ex2_ftz(q.x - M);
+              }
+            lse_s[t] = (t < p.R && l > 0.f) ? M + log2f(l) : INFINITY;
+          }
+        }
         named_bar_sync(1, NEPI);
       }
       // the MMA warp alternates accumulators continuously across items: tile k of the
@@ -343,7 +383,7 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
         if (lane == 0) mbar_arrive(&tm_empty[grp]);
 
         const int n0 = j * TC_TILE;
-        if (PASS == 1) {
+        if (p1) {
           if (t < p.R) {
             const int nv = min(vis - n0, TC_TILE);      // visible columns of this tile
             if (nv > 0) {
@@ -405,21 +445,38 @@ score_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant
       tiles_before += j1 - j0;
       // both groups meet here whatever happened; any failed wait stops every epilogue warp
       if (named_bar_or(2, NEPI, !ok)) { ok = false; break; }
-      if (PASS == 1) {
+      if (p1) {
         // merge the two groups' running stats of row t, then write the item's partial
         if (grp == 1) xch[t] = make_float2(m2, lsum);
         named_bar_sync(2, NEPI);
-        if (grp == 0 && t < p.R) {
+        if (grp == 0) {
           const float2 o = xch[t];
           const float M = fmaxf(m2, o.x);
           float l = 0.f;
           if (M != -INFINITY)
             l = (m2 == -INFINITY ? 0.f : lsum * ex2_ftz(m2 - M)) + (o.x == -INFINITY ? 0.f : o.y * ex2_ftz(o.x - M));
-          p.part[((size_t)s * p.nsplit + sp) * p.R + t] = make_float2(M, l);
+          if (PASS == 1) {
+            if (t < p.R) p.part[((size_t)s * p.nsplit + sp) * p.R + t] = make_float2(M, l);
+          } else {
+            // fused: this CTA's stats of row t go to slot `me` of every CTA in the cluster
+            // (every row, so the byte count each CTA expects is fixed)
+            if (!cl_waited) { cluster_wait(); cl_waited = true; }
+            const uint32_t me = cluster_rank();
+            float2* mine = xall + me * TC_ROWS + t;
+            for (int r = 0; r < p.nsplit; ++r) {
+              if (r == (int)me) *mine = make_float2(M, l);
+              else st_async_f32x2(map_to_rank(mine, (uint32_t)r), M, l, map_to_rank(xbar, (uint32_t)r));
+            }
+            if (t == 0) mbar_arrive_expect_tx(xbar, (uint32_t)((p.nsplit - 1) * TC_ROWS * 8));
+          }
         }
       }
+      }   // sweeps
     }
+    // fused: do not leave while other CTAs may still be sending into this one
+    if (PASS == 3 && grp == 0 && !x_waited) mbar_wait_cluster(xbar, 0);
   }
+  if (PASS == 3 && !cl_waited) cluster_wait();
 
   // the producer and MMA lanes drained their own operations above
   tc_fence_before();
@@ -504,10 +561,38 @@ inline bool make_map_3d(CUtensorMap* m, const void* base, int d, long long rows,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Can one cluster of k fused scoring CTAs be resident (k up to 16 needs a GPC that large)?
+template <int D>
+bool tc_cluster_fits(int k, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, bool> known;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = known.find({k, dev});
+  if (it != known.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(k);
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = k;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  const bool ok = cudaOccupancyMaxActiveClusters(&n, score_tc_kernel<D, 3>, &cfg) == cudaSuccess && n >= 1;
+  cudaGetLastError();
+  known[{k, dev}] = ok;
+  return ok;
+}
+
 template <int D>
 kvc_status tc_score_d(const kvc_shape* sh, const void* q_win, const void* k, const int32_t* chunk_end, int32_t C,
                       const float* row_lse, float* score, float2* part, float* lse2, void* keys_ws, int sms,
-                      cudaStream_t st, fail_fn fail, unsigned* launches) {
+                      cudaStream_t st, fail_fn fail, unsigned* launches, bool force_two_pass) {
   const int S = sh->n_slots, R = sh->G * sh->w, L = sh->L;
   const int N = chunk_end ? C : L;
   const void* kbase = k;
@@ -535,8 +620,6 @@ kvc_status tc_score_d(const kvc_shape* sh, const void* q_win, const void* k, con
   p.part = part;
   p.lse2 = lse2;
   p.score = score;
-  const int items = S * p.nsplit;
-  const int grid = std::min(items, sms);
   const size_t smem = TcSmem<D>::ALLOC;
   static bool attr_set[2][64] = {};
   int dev = 0;
@@ -546,9 +629,48 @@ kvc_status tc_score_d(const kvc_shape* sh, const void* q_win, const void* k, con
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(score_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "kvc_score: smem attribute: %s", cudaGetErrorString(e));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(score_tc_kernel<D, 3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(score_tc_kernel<D, 3>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "kvc_score: kernel attribute: %s", cudaGetErrorString(e));
     attr_set[di][dev] = true;
   }
+  // Fused (one launch: both passes and the row-normaliser merge inside slot clusters) when
+  // the clusters of k = SMs / S CTAs keep >= 3/4 of the SMs busy and every CTA has at least
+  // 8 key tiles per pass to amortise its setup and the exchange; pass 2 then re-reads keys
+  // that pass 1 just brought into L2.
+  if (!row_lse && !force_two_pass) {
+    int k = std::min(TC_MAX_CLUSTER, sms / std::max(S, 1));
+    k = std::min(k, p.tiles);
+    if (k >= 1) {
+      const int tpi = (p.tiles + k - 1) / k;
+      k = (p.tiles + tpi - 1) / tpi;               // no empty key range
+      if (4LL * S * k >= 3LL * sms && tpi >= 8 && tc_cluster_fits<D>(k, smem)) {
+        TcParams pf = p;
+        pf.tpi = tpi;
+        pf.nsplit = k;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(S * k);
+        cfg.blockDim = dim3(TC_THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = k;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, score_tc_kernel<D, 3>, mq, mk, pf);
+        if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "kvc_score: fused launch: %s", cudaGetErrorString(e));
+        ++*launches;
+        return KVC_OK;
+      }
+    }
+  }
+  const int items = S * p.nsplit;
+  const int grid = std::min(items, sms);
   if (!row_lse) {
     score_tc_kernel<D, 1><<<grid, TC_THREADS, smem, st>>>(mq, mk, p);
     score_lse2_merge<<<S, 128, 0, st>>>(part, p.nsplit, R, lse2);
@@ -564,10 +686,12 @@ kvc_status tc_score_d(const kvc_shape* sh, const void* q_win, const void* k, con
 
 inline kvc_status tc_score(const kvc_shape* sh, const void* q_win, const void* k, const int32_t* chunk_end, int32_t C,
                            const float* row_lse, float* score, float2* part, float* lse2, void* keys_ws, int sms,
-                           cudaStream_t st, fail_fn fail, unsigned* launches) {
+                           cudaStream_t st, fail_fn fail, unsigned* launches, bool force_two_pass) {
   if (sh->d == 128)
-    return tc_score_d<128>(sh, q_win, k, chunk_end, C, row_lse, score, part, lse2, keys_ws, sms, st, fail, launches);
-  return tc_score_d<64>(sh, q_win, k, chunk_end, C, row_lse, score, part, lse2, keys_ws, sms, st, fail, launches);
+    return tc_score_d<128>(sh, q_win, k, chunk_end, C, row_lse, score, part, lse2, keys_ws, sms, st, fail, launches,
+                           force_two_pass);
+  return tc_score_d<64>(sh, q_win, k, chunk_end, C, row_lse, score, part, lse2, keys_ws, sms, st, fail, launches,
+                        force_two_pass);
 }
 
 }  // namespace kvc

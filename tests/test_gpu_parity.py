@@ -405,6 +405,20 @@ def test_fused_append_decode_overflow_keeps_old_rows():
     kvc.kvc_get_status()
 
 
+def test_two_launch_scoring_on_fused_workloads():
+    """Workloads whose scoring runs fused in slot clusters by default pass the same checks
+    through the two-launch form (pass 1, merge, pass 2), forced here."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, KVC_SCORE_PATH="twopass")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        "-k", "llama8b_shape_small_context or chunk_small or llama8b_full_size or "
+                              "ragged_context_lengths or gqa_group_sizes or head_dims_and_dtypes or window_of_one"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
 def test_token_split_decode_on_few_slot_workloads():
     """Workloads with few slots decode through thread-block clusters by default; the
     token-range split (forced here) passes the same oracle checks."""
