@@ -340,3 +340,51 @@ def chunk_select_local(cscore, chunk_end, target_tokens: int, n_local: int):
     toks = (np.concatenate([np.arange(starts[c], ends[c] + 1) for c in chosen]).astype(np.int64)
             if chosen.size else np.zeros(0, dtype=np.int64))
     return toks, chosen
+
+
+# ---------------------------------------------------------------------------
+# decode-time chunk re-selection - ChunkLLM ICAC
+# ---------------------------------------------------------------------------
+def icac_decode(q_win, k, v, chunk_end, q_dec, k_dec, v_dec, boundary_steps, keep_frac: float,
+                n_local: int, G: int):
+    """ChunkLLM decode with re-selection at chunk boundaries (its Section 2.3: chunk
+    selection runs only when the current token closes a chunk - the Intra-Chunk
+    Attention Consistency pattern - and the selection holds until the next boundary).
+
+    One slot. The full cache (prompt plus every generated token) stays available;
+    the attended cache is the selected chunks plus the tokens generated since the
+    last selection. Step t appends token L + t to both, then attends over the
+    attended cache with q_dec[t]. If step t is in `boundary_steps`, token L + t
+    closes a chunk: the chunk list grows by it, every chunk is scored with the
+    single query q_dec[t] (the chunk scoring of `chunk_scores` with a window of
+    one), and the selection becomes `chunk_select_local` over all chunks with the
+    target ceil(keep_frac * (L + t + 1)) tokens - for the steps after t.
+
+    Returns (outputs [steps, G, d], selections: {step: token indices} at the start
+    and after every boundary step, keyed -1 for the prompt selection).
+    """
+    kf = np.concatenate([_f64(k), _f64(k_dec)], axis=0)
+    vf = np.concatenate([_f64(v), _f64(v_dec)], axis=0)
+    L = _f64(k).shape[0]
+    steps = _f64(q_dec).shape[0]
+    ends = [int(e) for e in np.asarray(chunk_end, dtype=np.int64)]
+    target = int(np.ceil(keep_frac * L))
+    cs = chunk_scores(q_win, kf[None, :L], L, np.asarray(ends))[0]
+    sel, _ = chunk_select_local(cs, np.asarray(ends), target, n_local)
+    sels = {-1: sel.copy()}
+    bset = set(int(b) for b in boundary_steps)
+    outs = np.zeros((steps, G, kf.shape[1]))
+    attended = list(sel)
+    for t in range(steps):
+        n = L + t + 1
+        attended.append(L + t)
+        idx = np.asarray(attended, dtype=np.int64)
+        q = _f64(q_dec[t])
+        outs[t] = decode_attention(q, kf[idx], vf[idx], [0, idx.size], [idx.size], G)
+        if t in bset:
+            ends.append(L + t)
+            cs = chunk_scores(q[:, None, :], kf[None, :n], n, np.asarray(ends))[0]
+            sel, _ = chunk_select_local(cs, np.asarray(ends), int(np.ceil(keep_frac * n)), n_local)
+            sels[t] = sel.copy()
+            attended = list(sel)
+    return outs, sels

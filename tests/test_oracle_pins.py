@@ -406,3 +406,79 @@ def test_chunk_select_local_reduces_and_forces():
     ends = np.array([2, 5, 9])
     toks, chosen = O.chunk_select_local(np.array([0.1, 0.2, 0.3]), ends, 1, 3)
     np.testing.assert_array_equal(toks, np.arange(10))
+
+
+# ---------------------------------------------------------------- ICAC re-selection (NEXT-1)
+def _attend(q, keys, vals):
+    """Plain softmax attention of each row of q over keys (numpy, fp64)."""
+    lg = q @ keys.T / np.sqrt(q.shape[1])
+    p = np.exp(lg - lg.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ vals
+
+
+def _icac_case(seed, L=60, steps=8, d=8, G=2, w=3):
+    r = _rng(seed)
+    k = r.standard_normal((L, d)); v = r.standard_normal((L, d))
+    qw = r.standard_normal((G, w, d))
+    qd = r.standard_normal((steps, G, d)); kd = r.standard_normal((steps, d)); vd = r.standard_normal((steps, d))
+    cuts = np.sort(r.choice(np.arange(L - 1), size=9, replace=False))
+    ends = np.concatenate([cuts, [L - 1]])
+    return k, v, qw, qd, kd, vd, ends
+
+
+def test_icac_keep_everything_is_full_attention():
+    """keep_frac = 1 keeps every chunk at every selection: each step is attention over
+    the whole prompt plus the generated tokens, whatever the boundaries."""
+    k, v, qw, qd, kd, vd, ends = _icac_case(401)
+    out, sels = O.icac_decode(qw, k, v, ends, qd, kd, vd, [1, 2, 5], 1.0, 0, 2)
+    for t in range(qd.shape[0]):
+        keys = np.concatenate([k, kd[:t + 1]]); vals = np.concatenate([v, vd[:t + 1]])
+        np.testing.assert_allclose(out[t], _attend(qd[t], keys, vals), rtol=1e-12, atol=1e-12)
+    for t in (1, 2, 5):
+        np.testing.assert_array_equal(sels[t], np.arange(k.shape[0] + t + 1))
+
+
+def test_icac_selection_timing_and_attended_sets():
+    """Brute force on explicit token sets: before any boundary the attended set is the
+    prompt selection plus the generated tokens; a boundary step still attends over the old
+    set, the next step over the new selection (which covers every token up to the boundary,
+    the closed chunk among its candidates) plus the tokens generated after it."""
+    k, v, qw, qd, kd, vd, ends = _icac_case(402)
+    L, steps = k.shape[0], qd.shape[0]
+    tb = 3
+    out, sels = O.icac_decode(qw, k, v, ends, qd, kd, vd, [tb], 0.5, 1, 2)
+    kf = np.concatenate([k, kd]); vf = np.concatenate([v, vd])
+    s0 = sels[-1]
+    for t in range(steps):
+        att = np.concatenate([s0, np.arange(L, L + t + 1)]) if t <= tb else \
+            np.concatenate([sels[tb], np.arange(L + tb + 1, L + t + 1)])
+        np.testing.assert_allclose(out[t], _attend(qd[t], kf[att], vf[att]), rtol=1e-12, atol=1e-12)
+    # the re-selection at tb: chunks are the prompt's plus [L, L + tb]; n_local = 1 keeps
+    # that newest chunk; at least half of the L + tb + 1 tokens are kept
+    new = sels[tb]
+    assert set(range(L, L + tb + 1)) <= set(new.tolist())
+    assert new.size >= math.ceil(0.5 * (L + tb + 1))
+    # and it is the chunk selection of the boundary query over those chunks (scores by
+    # direct softmax of q . chunk key over the visible chunks, summed over the group)
+    e2 = np.concatenate([ends, [L + tb]])
+    lg = qd[tb] @ kf[e2].T / np.sqrt(k.shape[1])
+    p = np.exp(lg - lg.max(axis=1, keepdims=True)); p /= p.sum(axis=1, keepdims=True)
+    toks, _ = O.chunk_select_local(p.sum(axis=0), e2, math.ceil(0.5 * (L + tb + 1)), 1)
+    np.testing.assert_array_equal(new, toks)
+
+
+def test_icac_query_picks_the_aligned_chunk():
+    """Two prompt chunks; the boundary query points at the first chunk's key and away
+    from the second's, so with room for one prompt chunk the re-selection keeps the first
+    (plus the closed generated chunk, which n_local = 1 forces)."""
+    d, G = 4, 1
+    k = np.zeros((8, d)); v = np.arange(8 * d, dtype=float).reshape(8, d)
+    k[3] = [5, 0, 0, 0]; k[7] = [-5, 0, 0, 0]           # chunk keys (last tokens of [0,3] and [4,7])
+    ends = np.array([3, 7])
+    qw = np.zeros((G, 1, d)); qw[0, 0] = [0, 1, 0, 0]     # prompt query: indifferent
+    qd = np.zeros((2, G, d)); qd[0, 0] = [1, 0, 0, 0]     # step 0 query favours chunk 0
+    kd = np.zeros((2, d)); vd = np.zeros((2, d))
+    out, sels = O.icac_decode(qw, k, v, ends, qd, kd, vd, [0], 0.5, 1, G)
+    # after step 0 (9 tokens, target 5): chunk [8] forced (1 token) + the best prompt chunk
+    np.testing.assert_array_equal(sels[0], np.array([0, 1, 2, 3, 8]))

@@ -14,6 +14,11 @@ describe:
                  (local window / special tokens / full cache).
 * ``chunk``    - 128K context with ChunkLLM-style chunk selection (chunk key =
                  key of the chunk's last token, keep top chunks totalling 48 %).
+* ``chunk_icac`` - the same with ChunkLLM's decode-time re-selection: whenever a
+                 generated token closes a chunk, the chunks are re-scored against
+                 that step's query and re-selected (16 most recent chunks always
+                 kept, as in ChunkLLM's long-generation setting). Not one of the
+                 five benchmark workloads.
 
 Nothing here computes any part of the method; this module only holds sizes.
 """
@@ -48,6 +53,8 @@ class Workload:
     special_frac: float = 0.04 # fastgen special-token set size as a fraction of L
     chunk_mean: float = 24.0   # chunk: mean of the Geometric chunk length
     keep_frac: float = 0.48    # chunk: fraction of tokens the kept chunks must reach
+    icac: bool = False         # chunk: re-select chunks at every generated chunk boundary (ChunkLLM ICAC)
+    n_local: int = 0           # chunk: most recent chunks always kept (ChunkLLM local chunks)
 
     # ---- derived sizes -------------------------------------------------
     @property
@@ -106,6 +113,9 @@ WORKLOADS = {
     "chunk": Workload(
         name="chunk", n_layers=1, batch=1, hq=32, hkv=8, d=128, L=131072, dtype="bf16",
         w=32, policy="chunk", steps=256, seed=5),
+    "chunk_icac": Workload(
+        name="chunk_icac", n_layers=1, batch=1, hq=32, hkv=8, d=128, L=131072, dtype="bf16",
+        w=32, policy="chunk", steps=256, seed=5, icac=True, n_local=16),
 }
 
 ORDER = ["tiny", "llama8b", "zigzag", "fastgen", "chunk"]

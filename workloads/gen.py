@@ -12,6 +12,7 @@ Draw order (fixed; every array comes from one torch.Generator seeded per workloa
   decode generator (seed + 1000) : q_dec [steps, nL*B*Hq, d], k_dec, v_dec [steps, nL*B*Hkv, d]
   host generator  (seed + 2000)  : fastgen policy per slot, special positions per batch row
   host generator  (seed + 3000)  : chunk lengths ~ Geometric(1/mean) on {1, 2, ...}
+  host generator  (seed + 4000)  : the same for the generated tokens (chunk_icac)
 
 All draws are fp32 N(0, 1) (or U for temperatures); bf16 workloads round the final
 fp32 values to the nearest bf16 (ties to even), so both sides read identical values.
@@ -142,3 +143,23 @@ def chunk_boundaries(wl: Workload) -> torch.Tensor:
             if pos >= wl.L - 1:
                 break
     return torch.tensor(ends, dtype=torch.int32)
+
+
+def decode_chunk_boundaries(wl: Workload) -> list:
+    """Decode steps whose generated token closes a chunk: the chunk process of
+    `chunk_boundaries` continued past the prompt (its last chunk ends at L - 1), with
+    lengths ~ Geometric(p = 1/mean) from its own generator. Step t appends position L + t."""
+    gh = _gen(wl.seed + 4000, "cpu")
+    p = 1.0 / wl.chunk_mean
+    log1mp = math.log1p(-p)
+    steps = []
+    pos = wl.L - 1
+    while True:
+        draw = torch.rand((256,), generator=gh, dtype=torch.float64)
+        lens = torch.floor(torch.log(1.0 - draw) / log1mp).to(torch.int64) + 1
+        for ln in lens.tolist():
+            pos += int(ln)
+            t = pos - wl.L
+            if t >= wl.steps:
+                return steps
+            steps.append(t)
