@@ -201,7 +201,11 @@ def cuda_arm(args, wl, rank, world, local_rank):
     kvc.library()
     wl_r = wl.scaled(seed=wl.seed + 100003 * rank)
     inp = make_inputs(wl_r, dev)
-    pipe = KvcPipeline(wl_r, inp)
+    bnd = None
+    if getattr(wl_r, "icac", False):
+        from workloads import decode_chunk_boundaries
+        bnd = decode_chunk_boundaries(wl_r)
+    pipe = KvcPipeline(wl_r, inp, decode_boundaries=bnd)
     stream = torch.cuda.current_stream()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)

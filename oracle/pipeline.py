@@ -79,11 +79,28 @@ def run_workload(inp, slots=None, steps=None, budgets=None, need_all_counts=True
                 res.sel[s] = O.special_indices(inp.special_mask[b].cpu().numpy())
             else:
                 res.sel[s] = O.full_indices(L)
+        elif wl.policy == "chunk" and getattr(wl, "icac", False):
+            # ChunkLLM decode-time re-selection: the prompt selection keeps n_local local
+            # chunks; the decode loop below re-selects at the generated chunk boundaries
+            toks, _ = O.chunk_select_local(score_of(s), inp.chunk_end.cpu().numpy(), wl.chunk_target, wl.n_local)
+            res.sel[s] = toks
         elif wl.policy == "chunk":
             toks, _ = O.chunk_select(score_of(s), inp.chunk_end.cpu().numpy(), wl.chunk_target)
             res.sel[s] = toks
         else:  # pragma: no cover
             raise ValueError(wl.policy)
+
+    if steps > 0 and wl.policy == "chunk" and getattr(wl, "icac", False):
+        from workloads import decode_chunk_boundaries
+        bnd = decode_chunk_boundaries(wl)
+        ce = inp.chunk_end.cpu().numpy()
+        for s in slots:
+            outs, _ = O.icac_decode(inp.q_win[s * G:(s + 1) * G], inp.k[s], inp.v[s], ce,
+                                    inp.q_dec[:steps, s * G:(s + 1) * G], inp.k_dec[:steps, s], inp.v_dec[:steps, s],
+                                    [b for b in bnd if b < steps], wl.keep_frac, wl.n_local, G)
+            for t in range(steps):
+                res.out[(t, s)] = outs[t]
+        return res
 
     if steps > 0:
         for s in slots:

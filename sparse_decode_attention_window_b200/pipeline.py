@@ -1,6 +1,11 @@
 """One workload through the C ABI: window scoring -> selection (-> ZigZagKV
 allocation) -> layout -> compaction, then per decode step append -> decode.
 
+With decode-time chunk re-selection (ChunkLLM's ICAC, Section 2.3) the full cache is
+kept as well: every step appends to it, and a step whose token closes a chunk re-scores
+all chunks with that step's query, re-selects them and re-compacts the attended cache
+from the full one - the same calls as the prompt's, over the grown chunk list.
+
 Host-side orchestration only: buffers are torch CUDA tensors allocated once,
 every step is a libkvc call on one stream.
 """
@@ -8,8 +13,10 @@ from __future__ import annotations
 
 import torch
 
+import math
+
 from . import (kvc_score, kvc_select, kvc_alloc_budgets, kvc_layout, kvc_compact, kvc_append, kvc_decode_attn,
-               kvc_append_decode,
+               kvc_append_decode, kvc_select_chunks,
                kvc_workspace_size, make_shape, KVC_WS_SCORE, KVC_WS_DECODE, KVC_POL_TOPB, KVC_POL_MASS_COUNT,
                KVC_POL_CHUNK)
 
@@ -22,9 +29,11 @@ class KvcPipeline:
     """Buffers and call sequence for one workload (see workloads.configs).
 
     `inp` is a workloads.Inputs whose tensors are on the target CUDA device.
+    `decode_boundaries`: for a chunk workload with `icac`, the decode steps whose token
+    closes a chunk (the chunk-boundary predictions the method receives).
     """
 
-    def __init__(self, wl, inp, device=None):
+    def __init__(self, wl, inp, device=None, decode_boundaries=None):
         self.wl = wl
         self.inp = inp
         dev = torch.device(device) if device is not None else inp.k.device
@@ -69,6 +78,45 @@ class KvcPipeline:
         self.vp = torch.empty((self.kp_rows, d), dtype=dt, device=dev)
         self.out = torch.empty((S * G, d), dtype=torch.float32, device=dev)
         self.ws_decode = torch.zeros(kvc_workspace_size(KVC_WS_DECODE, self.shape), dtype=torch.uint8, device=dev)
+        self.icac = bool(getattr(wl, "icac", False)) and wl.policy == "chunk"
+        if self.icac:
+            self._init_icac(decode_boundaries or [])
+
+    def _init_icac(self, boundaries):
+        wl, inp, dev = self.wl, self.inp, self.dev
+        S, G, d, L = wl.n_slots, wl.G, wl.d, wl.L
+        dt = inp.k.dtype
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.boundaries = sorted(int(b) for b in boundaries if 0 <= int(b) < wl.steps)
+        self.Lmax = _round16(L + wl.steps)
+        # the full cache: prompt keys/values plus every generated token, a packed layout
+        # with one Lmax-row region per slot
+        self.kf = torch.zeros((S, self.Lmax, d), dtype=dt, device=dev)
+        self.vf = torch.zeros((S, self.Lmax, d), dtype=dt, device=dev)
+        self.kf[:, :L].copy_(inp.k)
+        self.vf[:, :L].copy_(inp.v)
+        self.off_f = torch.arange(0, (S + 1) * self.Lmax, self.Lmax, dtype=torch.int64, device=dev)
+        self.cap_f = torch.full((S,), self.Lmax, **i32)
+        self.len_f = torch.full((S,), L, **i32)
+        # chunk list: the prompt's chunks, then one per boundary (token L + t closes it)
+        ends = inp.chunk_end.to(torch.int64).cpu().tolist() + [L + t for t in self.boundaries]
+        self.ends_all = torch.tensor(ends, **i32)
+        self.C0 = self.C
+        Cmax = len(ends)
+        self.shape_full = make_shape(S, G, d, self.Lmax, 1, wl.hkv, wl.batch, dt)   # k stride Lmax, one query row
+        self.score_f = torch.empty((S * Cmax,), dtype=torch.float32, device=dev)
+        self.ws_score_f = torch.zeros(kvc_workspace_size(KVC_WS_SCORE, self.shape_full, Cmax), dtype=torch.uint8,
+                                      device=dev)
+        # per boundary: the token target ceil(keep_frac * current length)
+        self.targets = torch.tensor([[math.ceil(wl.keep_frac * (L + t + 1))] * S for t in self.boundaries] or [[0] * S],
+                                    **i32)
+        self.prompt_target = torch.full((S,), wl.chunk_target, **i32)
+        # the attended cache and the selection can now hold any token of the full cache
+        self.max_sel = self.Lmax
+        self.idx = torch.empty((S, self.max_sel), **i32)
+        self.kp_rows = S * _round16(self.Lmax + wl.reserve)
+        self.kp = torch.empty((self.kp_rows, d), dtype=dt, device=dev)
+        self.vp = torch.empty((self.kp_rows, d), dtype=dt, device=dev)
 
     # ---- the hot path
     def score_step(self, stream=None):
@@ -90,6 +138,9 @@ class KvcPipeline:
         elif wl.policy == "fastgen":
             kvc_select(self.shape, None, self.policy, self.budget, self.idx, self.count,
                        special_mask=inp.special_mask, stream=stream)
+        elif wl.policy == "chunk" and self.icac:
+            kvc_select_chunks(self.shape, self.score, self.chunk_end, self.prompt_target, self.idx, self.count,
+                              n_local=wl.n_local, stream=stream)
         elif wl.policy == "chunk":
             kvc_select(self.shape, self.score, self.policy, self.budget, self.idx, self.count,
                        chunk_end=self.chunk_end, C=self.C, stream=stream)
@@ -97,6 +148,8 @@ class KvcPipeline:
             kvc_select(self.shape, self.score, self.policy, self.budget, self.idx, self.count, stream=stream)
 
     def compact_step(self, stream=None):
+        if self.icac:
+            self.len_f.fill_(self.wl.L)    # the full cache restarts from the prompt
         kvc_layout(self.count, self.wl.reserve, self.off, self.cap, stream=stream)
         kvc_compact(self.shape, self.inp.k, self.inp.v, self.idx, self.count, self.off, self.kp, self.vp, self.len,
                     stream=stream)
@@ -114,13 +167,38 @@ class KvcPipeline:
         k_new = inp.k_dec[t] if k_new is None else k_new
         v_new = inp.v_dec[t] if v_new is None else v_new
         out = self.out if out is None else out
+        if self.icac:
+            kvc_append(self.shape, k_new, v_new, self.off_f, self.cap_f, self.len_f, self.kf.view(-1, self.wl.d),
+                       self.vf.view(-1, self.wl.d), stream=stream)
         if fused:
             kvc_append_decode(self.shape, k_new, v_new, q, self.kp, self.vp, self.off, self.cap, self.len, out,
                               self.ws_decode, stream=stream)
         else:
             kvc_append(self.shape, k_new, v_new, self.off, self.cap, self.len, self.kp, self.vp, stream=stream)
             kvc_decode_attn(self.shape, q, self.kp, self.vp, self.off, self.len, out, self.ws_decode, stream=stream)
+        if self.icac and t in self.boundaries:
+            self.reselect_step(t, q, stream)
         return out
+
+    def reselect_step(self, t: int, q, stream=None):
+        """Token L + t closed a chunk: score every chunk with this step's query (a window
+        of one row over the chunk keys of the full cache), re-select and re-compact the
+        attended cache from the full cache, with room for the remaining steps."""
+        wl = self.wl
+        S, G, d = wl.n_slots, wl.G, wl.d
+        i = self.boundaries.index(t)
+        C = self.C0 + i + 1
+        n = wl.L + t + 1
+        ends = self.ends_all[:C]
+        score = self.score_f[:S * C].view(S, C)
+        kvc_score(self.shape_full, q.view(S * G, 1, d), self.kf, score, self.ws_score_f, chunk_end=ends, C=C,
+                  stream=stream)
+        shape_n = make_shape(S, G, d, n, 1, wl.hkv, wl.batch, self.kf.dtype)   # n tokens to choose from
+        kvc_select_chunks(shape_n, score, ends, self.targets[i], self.idx, self.count, n_local=wl.n_local,
+                          stream=stream)
+        kvc_layout(self.count, wl.steps - t - 1, self.off, self.cap, stream=stream)
+        kvc_compact(self.shape_full, self.kf, self.vf, self.idx, self.count, self.off, self.kp, self.vp, self.len,
+                    stream=stream)
 
     def run(self, steps=None, record=False, stream=None):
         self.compress(stream)

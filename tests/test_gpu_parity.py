@@ -3,6 +3,8 @@
 Small workloads are checked on every slot and step; the full-size workloads run
 in the same launch configuration the benchmark times and are checked on sampled
 slots and steps (the oracle computes them one by one)."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -531,3 +533,91 @@ def test_chunk_selection_with_local_chunks(n_local):
                        if any(c < C - nl for c in cid) else np.zeros(0, np.int64),
                        free_sc, ce[: C - nl], wl.chunk_target - int((np.diff(np.concatenate([[-1], ce]))[C - nl:]).sum()),
                        f"slot {s}")
+
+
+def _check_local_chunk_selection(got, ref_sc, ce, target, n_local, what):
+    """GPU tokens of a selection with local chunks vs the oracle's rule (ties tolerated)."""
+    C = len(ce)
+    toks, _ = O.chunk_select_local(ref_sc, ce, target, n_local)
+    if np.array_equal(got, toks):
+        return
+    nl = min(n_local, C)
+    cid = np.unique(np.searchsorted(ce, got, side="left"))
+    assert set(range(C - nl, C)) <= set(cid.tolist()), f"{what}: local chunks missing"
+    starts = np.concatenate([[0], ce[:-1] + 1])
+    lens = ce - starts + 1
+    have = int(lens[C - nl:].sum())
+    free = [c for c in cid if c < C - nl]
+    free_toks = (np.concatenate([np.arange(starts[c], ce[c] + 1) for c in free]) if free
+                 else np.zeros(0, np.int64))
+    if have >= target:
+        assert not free, f"{what}: local chunks reach the target, nothing else may be kept"
+        return
+    P.check_chunks(free_toks, ref_sc[: C - nl], ce[: C - nl], target - have, what)
+
+
+@pytest.mark.parametrize("n_local", [0, 4])
+def test_chunk_icac_reselection_matches_oracle(n_local):
+    """ChunkLLM decode-time re-selection (NEXT-1): at every step whose token closes a chunk
+    the chunks are re-scored with that step's query, re-selected and the attended cache is
+    re-compacted from the full cache. Each GPU selection is checked against the oracle's
+    rule on the oracle's chunk scores (ties tolerated); each step's output against fp64
+    attention over the GPU's attended set; with no tie, the whole run equals icac_decode."""
+    from workloads import decode_chunk_boundaries
+    from sparse_decode_attention_window_b200.pipeline import KvcPipeline
+    import sparse_decode_attention_window_b200 as kvc
+    from dataclasses import replace
+    wl = get("chunk_icac").scaled(L=3000, steps=40, chunk_mean=8.0, n_local=n_local)
+    inp = make_inputs(wl, "cpu")
+    dinp = replace(inp, **{f: getattr(inp, f).cuda() for f in ("q_win", "k", "v", "q_dec", "k_dec", "v_dec",
+                                                                 "chunk_end")})
+    bnd = decode_chunk_boundaries(wl)
+    assert len(bnd) >= 3
+    pipe = KvcPipeline(wl, dinp, decode_boundaries=bnd)
+    pipe.compress()
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    S, G, L = wl.n_slots, wl.G, wl.L
+    ce0 = _np(dinp.chunk_end).astype(np.int64)
+    kf = np.concatenate([O._f64(inp.k), O._f64(inp.k_dec).transpose(1, 0, 2)], axis=1)   # [S, L + steps, d]
+    vf = np.concatenate([O._f64(inp.v), O._f64(inp.v_dec).transpose(1, 0, 2)], axis=1)
+    sel = {}
+    for s in range(S):
+        got = _np(pipe.idx[s, :int(pipe.count[s])]).astype(np.int64)
+        ref_sc = O.chunk_scores(inp.q_win[s * G:(s + 1) * G], inp.k[s:s + 1], L, ce0)[0]
+        _check_local_chunk_selection(got, ref_sc, ce0, wl.chunk_target, n_local, f"prompt slot {s}")
+        sel[s] = list(got)
+    ends = list(ce0)
+    exact = True
+    gpu_out = []
+    for t in range(wl.steps):
+        out = _np(pipe.decode_step(t)).copy()
+        gpu_out.append(out)
+        torch.cuda.synchronize()
+        kvc.kvc_get_status()
+        for s in range(S):
+            sel[s].append(L + t)
+            idx = np.asarray(sel[s], dtype=np.int64)
+            q = O._f64(inp.q_dec[t, s * G:(s + 1) * G])
+            ref = O.decode_attention(q, kf[s][idx], vf[s][idx], [0, idx.size], [idx.size], G)
+            P.check_out(out[s * G:(s + 1) * G], ref, "bf16", f"step {t} slot {s}")
+        if t in bnd:
+            ends.append(L + t)
+            e = np.asarray(ends, dtype=np.int64)
+            n = L + t + 1
+            target = math.ceil(wl.keep_frac * n)
+            for s in range(S):
+                got = _np(pipe.idx[s, :int(pipe.count[s])]).astype(np.int64)
+                q = O._f64(inp.q_dec[t, s * G:(s + 1) * G])
+                ref_sc = O.chunk_scores(q[:, None, :], kf[s][None, :n], n, e)[0]
+                _check_local_chunk_selection(got, ref_sc, e, target, n_local, f"boundary step {t} slot {s}")
+                toks, _ = O.chunk_select_local(ref_sc, e, target, n_local)
+                exact = exact and np.array_equal(got, toks)
+                sel[s] = list(got)
+                assert int(pipe.len[s]) == got.size
+    if exact:
+        for s in range(0, S, 3):
+            outs, _ = O.icac_decode(inp.q_win[s * G:(s + 1) * G], inp.k[s], inp.v[s], ce0, inp.q_dec[:, s * G:(s + 1) * G],
+                                    inp.k_dec[:, s], inp.v_dec[:, s], bnd, wl.keep_frac, n_local, G)
+            for t in range(wl.steps):
+                P.check_out(gpu_out[t][s * G:(s + 1) * G], outs[t], "bf16", f"icac_decode step {t} slot {s}")
