@@ -241,6 +241,22 @@ kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const 
                                    int64_t kp_rows, float* out, cudaStream_t stream);
 
 /*
+ * kvc_append_window - kvc_append with sliding-window eviction (the local-window variant
+ *   of FastGen's local heads - the policy keeps the most recent tokens - applied while
+ *   decoding): a slot with window[s] > 0 whose cache already holds window[s] rows keeps
+ *   exactly those rows; the new token overwrites row head[s] (the oldest) and head[s]
+ *   advances cyclically, len[s] unchanged. Every other slot appends at row len[s] and
+ *   increments len[s] (overflow past cap[s] is flagged, the row is not written).
+ *   Decode attention does not depend on the order of a slot's rows, so kvc_decode_attn
+ *   over [off[s], off[s] + len[s]) sees exactly the window. Compaction stores a local
+ *   slot's rows oldest first, so head[s] starts at 0.
+ *   k_new, v_new [S, d]; window [S] int32 (0: no eviction); head [S] int32, in/out.
+ */
+kvc_status kvc_append_window(const kvc_shape* shape, const void* k_new, const void* v_new, const int64_t* off,
+                             const int32_t* cap, int32_t* len, const int32_t* window, int32_t* head,
+                             void* kp, void* vp, int64_t kp_rows, cudaStream_t stream);
+
+/*
  * kvc_select_chunks - ChunkLLM chunk selection with always-kept local chunks (ChunkLLM
  *   Section 3.2 keeps the 15 or 16 most recent chunks): for every slot, the last
  *   n_local chunks are kept, then the other chunks in descending chunk-score order

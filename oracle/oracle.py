@@ -388,3 +388,11 @@ def icac_decode(q_win, k, v, chunk_end, q_dec, k_dec, v_dec, boundary_steps, kee
             sels[t] = sel.copy()
             attended = list(sel)
     return outs, sels
+
+
+def sliding_local_indices(L: int, t: int, window: int) -> np.ndarray:
+    """FastGen local heads with eviction while decoding: a local head attends to the most
+    recent `window` tokens of the sequence, so at decode step t (token L + t appended) it
+    keeps positions [L + t + 1 - window, L + t] (the local-window variant of the policy)."""
+    n = int(L) + int(t) + 1
+    return np.arange(max(0, n - int(window)), n, dtype=np.int64)

@@ -102,6 +102,19 @@ def run_workload(inp, slots=None, steps=None, budgets=None, need_all_counts=True
                 res.out[(t, s)] = outs[t]
         return res
 
+    if steps > 0 and wl.policy == "fastgen" and getattr(wl, "local_sliding", False):
+        # local heads keep exactly their last local_window tokens while decoding
+        for s in slots:
+            kf = np.concatenate([O._f64(inp.k[s]), O._f64(inp.k_dec[:steps, s])], axis=0)
+            vf = np.concatenate([O._f64(inp.v[s]), O._f64(inp.v_dec[:steps, s])], axis=0)
+            local = int(inp.policy[s]) == LOCAL
+            for t in range(steps):
+                idx = (O.sliding_local_indices(L, t, wl.local_window) if local
+                       else np.concatenate([res.sel[s], np.arange(L, L + t + 1)]))
+                q = O._f64(inp.q_dec[t, s * G:(s + 1) * G])
+                res.out[(t, s)] = O.decode_attention(q, kf[idx], vf[idx], [0, idx.size], [idx.size], G)
+        return res
+
     if steps > 0:
         for s in slots:
             idx = res.sel[s]

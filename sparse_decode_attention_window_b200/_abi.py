@@ -20,6 +20,7 @@ KVC_WS_SCORE, KVC_WS_SELECT, KVC_WS_DECODE = 0, 1, 2
 
 # every symbol the header declares
 EXPORTS = ["kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout", "kvc_compact", "kvc_append",
+           "kvc_append_window",
            "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_last_error", "kvc_version",
            "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_select_chunks",
            "kvc_retained_mass", "kvc_profile_heads"]
@@ -59,6 +60,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "kvc_layout": (i32, [vp, i32, i32, vp, vp, vp]),
         "kvc_compact": (i32, [sh, vp, vp, vp, i32, vp, vp, vp, vp, i64, vp, vp]),
         "kvc_append": (i32, [sh, vp, vp, vp, vp, vp, vp, vp, i64, vp]),
+        "kvc_append_window": (i32, [sh, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp]),
         "kvc_decode_attn": (i32, [sh, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
         "kvc_workspace_size": (sz, [ctypes.c_int, sh, i32]),
         "kvc_get_status": (i32, [vp]),

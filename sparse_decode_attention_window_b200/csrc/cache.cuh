@@ -115,6 +115,35 @@ __global__ void append_kernel(const uint4* __restrict__ k_new, const uint4* __re
   }
 }
 
+// ---------------------------------------------------------------- append with a sliding window
+// grid S, block TPR. A slot with window[s] > 0 that already holds window[s] rows keeps
+// holding them: the new token overwrites row head[s] (the oldest) and head[s] advances
+// cyclically. Any other slot appends as append_kernel. Attention over a slot's rows does
+// not depend on their order, so the window's rows can stay a ring.
+__global__ void append_window_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                     const int64_t* __restrict__ off, const int32_t* __restrict__ cap,
+                                     int32_t* __restrict__ len, const int32_t* __restrict__ window,
+                                     int32_t* __restrict__ head, uint4* __restrict__ kp, uint4* __restrict__ vp,
+                                     int64_t kp_rows, int tpr) {
+  const int s = blockIdx.x;
+  const int n = len[s], w = window[s];
+  const bool ring = w > 0 && n >= w;
+  const int h = ring ? head[s] : 0;
+  const int row = ring ? h : n;
+  const bool ok = n >= 0 && row >= 0 && row < cap[s] && (!ring || h < w) && off[s] + row < kp_rows;
+  if (ok) {
+    const size_t dst = ((size_t)off[s] + row) * tpr + threadIdx.x;
+    kp[dst] = k_new[(size_t)s * tpr + threadIdx.x];
+    vp[dst] = v_new[(size_t)s * tpr + threadIdx.x];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!ok) kvc_flag(KVC_DEVERR_APPEND_OVERFLOW);
+    else if (ring) head[s] = h + 1 == w ? 0 : h + 1;
+    else len[s] = n + 1;
+  }
+}
+
 // ---------------------------------------------------------------- chunk keys
 // kc[s][c] = k[s][chunk_end[c]] (ChunkLLM Eq. 3: a chunk is keyed by its last token).
 __global__ void gather_rows_kernel(const uint4* __restrict__ k, const int32_t* __restrict__ rows, int C, int L,

@@ -670,6 +670,23 @@ kvc_status kvc_compact(const kvc_shape* shape, const void* k, const void* v, con
   return check_launch("kvc_compact");
 }
 
+kvc_status kvc_append_window(const kvc_shape* shape, const void* k_new, const void* v_new, const int64_t* off,
+                             const int32_t* cap, int32_t* len, const int32_t* window, int32_t* head, void* kp,
+                             void* vp, int64_t kp_rows, cudaStream_t stream) {
+  kvc_status rc = check_shape(shape, false);
+  if (rc != KVC_OK) return rc;
+  if (!k_new || !v_new || !off || !cap || !len || !window || !head || !kp || !vp)
+    return fail(KVC_ERR_INVALID_ARG, "kvc_append_window: NULL pointer argument");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kp) || !aligned16(vp))
+    return fail(KVC_ERR_INVALID_ARG, "kvc_append_window: buffers must be 16-byte aligned");
+  const int tpr = (int)(shape->d * esize(shape->dtype) / 16);
+  kvc::append_window_kernel<<<shape->n_slots, tpr, 0, stream>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), off, cap, len, window, head,
+      static_cast<uint4*>(kp), static_cast<uint4*>(vp), kp_rows, tpr);
+  count_launches(1);
+  return check_launch("kvc_append_window");
+}
+
 kvc_status kvc_append(const kvc_shape* shape, const void* k_new, const void* v_new, const int64_t* off,
                       const int32_t* cap, int32_t* len, void* kp, void* vp, int64_t kp_rows, cudaStream_t stream) {
   kvc_status rc = check_shape(shape, false);

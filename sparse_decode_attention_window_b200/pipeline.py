@@ -16,7 +16,7 @@ import torch
 import math
 
 from . import (kvc_score, kvc_select, kvc_alloc_budgets, kvc_layout, kvc_compact, kvc_append, kvc_decode_attn,
-               kvc_append_decode, kvc_select_chunks,
+               kvc_append_decode, kvc_select_chunks, kvc_append_window, KVC_POL_LOCAL,
                kvc_workspace_size, make_shape, KVC_WS_SCORE, KVC_WS_DECODE, KVC_POL_TOPB, KVC_POL_MASS_COUNT,
                KVC_POL_CHUNK)
 
@@ -81,6 +81,11 @@ class KvcPipeline:
         self.icac = bool(getattr(wl, "icac", False)) and wl.policy == "chunk"
         if self.icac:
             self._init_icac(decode_boundaries or [])
+        # FastGen local heads that keep evicting while decoding: their rows form a ring
+        self.sliding = bool(getattr(wl, "local_sliding", False)) and wl.policy == "fastgen"
+        if self.sliding:
+            self.window = torch.where(inp.policy.to(dev) == KVC_POL_LOCAL, wl.local_window, 0).to(torch.int32)
+            self.head = torch.zeros((S,), **i32)
 
     def _init_icac(self, boundaries):
         wl, inp, dev = self.wl, self.inp, self.dev
@@ -150,6 +155,8 @@ class KvcPipeline:
     def compact_step(self, stream=None):
         if self.icac:
             self.len_f.fill_(self.wl.L)    # the full cache restarts from the prompt
+        if self.sliding:
+            self.head.zero_()              # compaction stores a local head's window oldest first
         kvc_layout(self.count, self.wl.reserve, self.off, self.cap, stream=stream)
         kvc_compact(self.shape, self.inp.k, self.inp.v, self.idx, self.count, self.off, self.kp, self.vp, self.len,
                     stream=stream)
@@ -170,7 +177,12 @@ class KvcPipeline:
         if self.icac:
             kvc_append(self.shape, k_new, v_new, self.off_f, self.cap_f, self.len_f, self.kf.view(-1, self.wl.d),
                        self.vf.view(-1, self.wl.d), stream=stream)
-        if fused:
+        if self.sliding:
+            # append (a full local window overwrites its oldest row), then decode
+            kvc_append_window(self.shape, k_new, v_new, self.off, self.cap, self.len, self.window, self.head,
+                              self.kp, self.vp, stream=stream)
+            kvc_decode_attn(self.shape, q, self.kp, self.vp, self.off, self.len, out, self.ws_decode, stream=stream)
+        elif fused:
             kvc_append_decode(self.shape, k_new, v_new, q, self.kp, self.vp, self.off, self.cap, self.len, out,
                               self.ws_decode, stream=stream)
         else:

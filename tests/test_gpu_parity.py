@@ -621,3 +621,33 @@ def test_chunk_icac_reselection_matches_oracle(n_local):
                                     inp.k_dec[:, s], inp.v_dec[:, s], bnd, wl.keep_frac, n_local, G)
             for t in range(wl.steps):
                 P.check_out(gpu_out[t][s * G:(s + 1) * G], outs[t], "bf16", f"icac_decode step {t} slot {s}")
+
+
+def test_fastgen_sliding_local_window_matches_oracle():
+    """NEXT-3: FastGen local heads keep exactly their most recent window while decoding
+    (kvc_append_window overwrites the oldest row once the window is full); every other
+    head keeps its selection plus all appended tokens. Enough steps to wrap the ring
+    twice; every step of every slot against the oracle."""
+    import sparse_decode_attention_window_b200 as kvc
+    from sparse_decode_attention_window_b200.pipeline import KvcPipeline
+    from oracle.pipeline import run_workload
+    from dataclasses import replace
+    wl = get("fastgen_sliding").scaled(batch=2, L=1500, local_window=48, steps=110)
+    inp = make_inputs(wl, "cpu")
+    dinp = replace(inp, **{f: (getattr(inp, f).cuda() if getattr(inp, f) is not None else None)
+                           for f in ("q_win", "k", "v", "q_dec", "k_dec", "v_dec", "policy", "special_mask")})
+    assert (inp.policy == POL_LOCAL).any()
+    pipe = KvcPipeline(wl, dinp)
+    pipe.compress()
+    outs = []
+    for t in range(wl.steps):
+        outs.append(_np(pipe.decode_step(t)).copy())
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    ref = run_workload(inp)
+    G = wl.G
+    for s in range(wl.n_slots):
+        if int(inp.policy[s]) == POL_LOCAL:
+            assert int(pipe.len[s]) == wl.local_window
+        for t in range(wl.steps):
+            P.check_out(outs[t][s * G:(s + 1) * G], ref.out[(t, s)], "bf16", f"step {t} slot {s}")

@@ -482,3 +482,13 @@ def test_icac_query_picks_the_aligned_chunk():
     out, sels = O.icac_decode(qw, k, v, ends, qd, kd, vd, [0], 0.5, 1, G)
     # after step 0 (9 tokens, target 5): chunk [8] forced (1 token) + the best prompt chunk
     np.testing.assert_array_equal(sels[0], np.array([0, 1, 2, 3, 8]))
+
+
+def test_sliding_local_indices_are_the_last_window():
+    """The local head's attended set after step t: exactly the last `window` positions of
+    the grown sequence (all of them while the sequence is shorter), brute-forced."""
+    for L, W in ((10, 4), (3, 8), (100, 100), (50, 1)):
+        for t in range(6):
+            got = O.sliding_local_indices(L, t, W)
+            seq = list(range(L + t + 1))
+            np.testing.assert_array_equal(got, np.array(seq[-W:] if W <= len(seq) else seq))

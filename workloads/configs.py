@@ -19,6 +19,8 @@ describe:
                  that step's query and re-selected (16 most recent chunks always
                  kept, as in ChunkLLM's long-generation setting). Not one of the
                  five benchmark workloads.
+* ``fastgen_sliding`` - fastgen whose local heads also evict while decoding: each keeps
+                 exactly its most recent 256 tokens. Not one of the five benchmark workloads.
 
 Nothing here computes any part of the method; this module only holds sizes.
 """
@@ -55,6 +57,7 @@ class Workload:
     keep_frac: float = 0.48    # chunk: fraction of tokens the kept chunks must reach
     icac: bool = False         # chunk: re-select chunks at every generated chunk boundary (ChunkLLM ICAC)
     n_local: int = 0           # chunk: most recent chunks always kept (ChunkLLM local chunks)
+    local_sliding: bool = False  # fastgen: local heads keep only their last local_window tokens while decoding
 
     # ---- derived sizes -------------------------------------------------
     @property
@@ -113,6 +116,9 @@ WORKLOADS = {
     "chunk": Workload(
         name="chunk", n_layers=1, batch=1, hq=32, hkv=8, d=128, L=131072, dtype="bf16",
         w=32, policy="chunk", steps=256, seed=5),
+    "fastgen_sliding": Workload(
+        name="fastgen_sliding", n_layers=1, batch=8, hq=32, hkv=8, d=128, L=16384, dtype="bf16",
+        w=0, policy="fastgen", steps=512, seed=4, local_sliding=True),
     "chunk_icac": Workload(
         name="chunk_icac", n_layers=1, batch=1, hq=32, hkv=8, d=128, L=131072, dtype="bf16",
         w=32, policy="chunk", steps=256, seed=5, icac=True, n_local=16),
