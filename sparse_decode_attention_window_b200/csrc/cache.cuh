@@ -94,6 +94,115 @@ __global__ void __launch_bounds__(256, 4) compact_kernel(const uint4* __restrict
   }
 }
 
+// ---------------------------------------------------------------- compaction, one wave
+// One CTA per (SM x 4), each owning the contiguous packed rows [r0, r1). Its dependent
+// round trips to memory are few and fixed: warp 0 finds the slots of r0 and r1 - 1 with
+// two 32-wide probes of off[]; the CTA stages those slots' offsets and counts in shared
+// memory (up to CP_MAX_SLOTS, else a chunk-local binary search in global memory); then,
+// 256 rows at a time, every thread resolves one row's source (one coalesced idx load)
+// and the CTA copies the chunk's K and V rows with 16-byte accesses, CP_UNROLL rows in
+// flight per row group.
+constexpr int CP_THREADS = 256;
+constexpr int CP_MAX_SLOTS = 512;
+constexpr int CP_UNROLL = 4;
+
+// last s in [0, S) with off[s] <= x, by two rounds of 32 probes (one warp)
+KVC_DEV int warp_slot_search(const int64_t* __restrict__ off, int S, long long x) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, n = S;
+  while (n > 1) {
+    const int step = (n + 31) / 32;
+    const int i = lo + lane * step;
+    const bool le = i < lo + n && off[i] <= x;
+    const unsigned m = __ballot_sync(0xffffffffu, le);
+    const int best = m ? 31 - __clz(m) : 0;
+    lo = lo + best * step;
+    n = min(step, S - lo);
+  }
+  return lo;
+}
+
+template <int TPR>
+__global__ void __launch_bounds__(CP_THREADS, 4) compact_wave_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, const int32_t* __restrict__ idx, int max_sel,
+    const int32_t* __restrict__ count, const int64_t* __restrict__ off, int S, int L, uint4* __restrict__ kp,
+    uint4* __restrict__ vp, int64_t kp_rows, int32_t* __restrict__ len) {
+  __shared__ long long s_off[CP_MAX_SLOTS + 1];
+  __shared__ int s_cnt[CP_MAX_SLOTS];
+  __shared__ long long src_row[CP_THREADS];   // source row s * L + j, or -1: not written
+  __shared__ int s_first_sh, s_last_sh;
+  const int tid = threadIdx.x;
+  for (long long s = (long long)blockIdx.x * blockDim.x + tid; s < S; s += (long long)gridDim.x * blockDim.x)
+    len[s] = min(max(count[s], 0), max_sel);
+  const long long total = off[S];
+  const long long r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
+  if (r0 >= r1) return;
+  if (tid < 32) {
+    const int a = warp_slot_search(off, S, r0);
+    const int b = warp_slot_search(off, S, r1 - 1);
+    if (tid == 0) { s_first_sh = a; s_last_sh = b; }
+  }
+  __syncthreads();
+  const int s_first = s_first_sh, ns = s_last_sh - s_first_sh + 1;
+  const bool staged = ns <= CP_MAX_SLOTS;
+  if (staged) {
+    for (int i = tid; i <= ns; i += blockDim.x) s_off[i] = off[s_first + i];
+    for (int i = tid; i < ns; i += blockDim.x) s_cnt[i] = min(count[s_first + i], max_sel);
+  }
+  __syncthreads();
+  constexpr int GROUPS = CP_THREADS / TPR;
+  const int part = tid % TPR, grp = tid / TPR;
+  for (long long base = r0; base < r1; base += CP_THREADS) {
+    // resolve one row per thread
+    const long long g = base + tid;
+    long long src = -1;
+    if (g < r1) {
+      int lo, hi;
+      if (staged) { lo = 0; hi = ns - 1; } else { lo = s_first; hi = s_first + ns - 1; }
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const long long om = staged ? s_off[mid] : off[mid];
+        if (om <= g) lo = mid; else hi = mid - 1;
+      }
+      const int s = staged ? s_first + lo : lo;
+      const long long r = g - (staged ? s_off[lo] : off[s]);
+      const int cnt = staged ? s_cnt[lo] : min(count[s], max_sel);
+      if (r < cnt) {
+        const int j = idx[(size_t)s * max_sel + r];
+        if (j < 0 || j >= L || g >= kp_rows) kvc_flag(KVC_DEVERR_INDEX_RANGE);
+        else src = (long long)s * L + j;
+      }
+    }
+    src_row[tid] = src;
+    __syncthreads();
+    const int nrows = (int)min((long long)CP_THREADS, r1 - base);
+    for (int i0 = grp; i0 < nrows; i0 += GROUPS * CP_UNROLL) {
+      uint4 kr[CP_UNROLL], vr[CP_UNROLL];
+      long long dst[CP_UNROLL];
+#pragma unroll
+      for (int u = 0; u < CP_UNROLL; ++u) {
+        const int i = i0 + u * GROUPS;
+        dst[u] = -1;
+        if (i < nrows) {
+          const long long sr = src_row[i];
+          if (sr >= 0) {
+            kr[u] = __ldg(k + (size_t)sr * TPR + part);
+            vr[u] = __ldg(v + (size_t)sr * TPR + part);
+            dst[u] = (base + i) * TPR + part;
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < CP_UNROLL; ++u)
+        if (dst[u] >= 0) {
+          kp[dst[u]] = kr[u];
+          vp[dst[u]] = vr[u];
+        }
+    }
+    __syncthreads();   // src_row is reused by the next chunk
+  }
+}
+
 // ---------------------------------------------------------------- append
 // grid S, block TPR: row off[s] + len[s] <- the new token; len[s] += 1.
 __global__ void append_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,

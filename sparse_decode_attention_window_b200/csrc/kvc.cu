@@ -127,6 +127,15 @@ bool force_two_pass_score() {
   return v;
 }
 
+// KVC_COMPACT_PATH=grid keeps the grid-stride compaction kernel (cross-checks); read once.
+bool force_old_compact() {
+  static const bool v = [] {
+    const char* e = getenv("KVC_COMPACT_PATH");
+    return e && strcmp(e, "grid") == 0;
+  }();
+  return v;
+}
+
 // KVC_DECODE_PATH=simt routes bf16 decode to the CUDA-core kernel (cross-checks); read once.
 bool force_simt_decode() {
   static const bool v = [] {
@@ -652,19 +661,33 @@ kvc_status kvc_compact(const kvc_shape* shape, const void* k, const void* v, con
   DevInfo* di = nullptr;
   if ((rc = dev_info(&di)) != KVC_OK) return rc;
   const int tpr = (int)(shape->d * esize(shape->dtype) / 16);
-  const int blocks = di->sms * 8;
   const uint4* k4 = static_cast<const uint4*>(k);
   const uint4* v4 = static_cast<const uint4*>(v);
   uint4* kp4 = static_cast<uint4*>(kp);
   uint4* vp4 = static_cast<uint4*>(vp);
-  switch (tpr) {
-    case 8: kvc::compact_kernel<8, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, shape->n_slots,
-                                                                   shape->L, kp4, vp4, kp_rows, len); break;
-    case 16: kvc::compact_kernel<16, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, shape->n_slots,
-                                                                     shape->L, kp4, vp4, kp_rows, len); break;
-    case 32: kvc::compact_kernel<32, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, shape->n_slots,
-                                                                     shape->L, kp4, vp4, kp_rows, len); break;
-    default: return fail(KVC_ERR_UNSUPPORTED, "kvc_compact: row of %d bytes", tpr * 16);
+  const int S = shape->n_slots, L = shape->L;
+  if (!force_old_compact()) {
+    const int blocks = di->sms * 4;   // one wave at four CTAs per SM
+    switch (tpr) {
+      case 8: kvc::compact_wave_kernel<8><<<blocks, kvc::CP_THREADS, 0, stream>>>(k4, v4, idx, max_sel, count, off, S,
+                                                                                  L, kp4, vp4, kp_rows, len); break;
+      case 16: kvc::compact_wave_kernel<16><<<blocks, kvc::CP_THREADS, 0, stream>>>(k4, v4, idx, max_sel, count, off,
+                                                                                    S, L, kp4, vp4, kp_rows, len); break;
+      case 32: kvc::compact_wave_kernel<32><<<blocks, kvc::CP_THREADS, 0, stream>>>(k4, v4, idx, max_sel, count, off,
+                                                                                    S, L, kp4, vp4, kp_rows, len); break;
+      default: return fail(KVC_ERR_UNSUPPORTED, "kvc_compact: row of %d bytes", tpr * 16);
+    }
+  } else {
+    const int blocks = di->sms * 8;
+    switch (tpr) {
+      case 8: kvc::compact_kernel<8, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, S, L, kp4, vp4,
+                                                                     kp_rows, len); break;
+      case 16: kvc::compact_kernel<16, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, S, L, kp4,
+                                                                       vp4, kp_rows, len); break;
+      case 32: kvc::compact_kernel<32, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, S, L, kp4,
+                                                                       vp4, kp_rows, len); break;
+      default: return fail(KVC_ERR_UNSUPPORTED, "kvc_compact: row of %d bytes", tpr * 16);
+    }
   }
   count_launches(1);
   return check_launch("kvc_compact");

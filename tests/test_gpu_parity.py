@@ -407,6 +407,19 @@ def test_fused_append_decode_overflow_keeps_old_rows():
     kvc.kvc_get_status()
 
 
+def test_grid_stride_compaction_on_workloads():
+    """The grid-stride compaction kernel (forced here; the one-wave kernel is the default)
+    gives the same bit-exact packed caches."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, KVC_COMPACT_PATH="grid")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        "-k", "llama8b_shape_small_context or zigzag_small or fastgen_small or chunk_small"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
 def test_two_launch_scoring_on_fused_workloads():
     """Workloads whose scoring runs fused in slot clusters by default pass the same checks
     through the two-launch form (pass 1, merge, pass 2), forced here."""
