@@ -316,7 +316,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   // the grid, and the lengths are near uniform (the same test in every CTA)
   const bool per_slot = ksz >= 2 && (long long)S * ksz <= nC && 4LL * S * ksz >= 3LL * nC &&
                         4LL * (long long)max_len_sh * S <= 5LL * N;
-  const int my_cluster = c / (ksz > 0 ? ksz : 1);
+  const int my_cluster = per_slot ? (int)((unsigned)c / (unsigned)ksz) : c;
   const bool in_slot_cluster = per_slot && my_cluster < S;
   int nE = 0;
   bool active = false;
@@ -332,9 +332,16 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     }
     active = b1 > b0;
   } else if (in_slot_cluster) {
-    const long long r = (long long)cluster_rank(), ns = P[my_cluster + 1] - P[my_cluster];
-    b0 = P[my_cluster] + r * ns / ksz;
-    b1 = P[my_cluster] + (r + 1) * ns / ksz;
+    const long long ns = P[my_cluster + 1] - P[my_cluster];
+    const unsigned r = cluster_rank(), k = (unsigned)ksz;
+    if (ns < (1LL << 27)) {            // 32-bit arithmetic (a 64-bit division costs hundreds of cycles)
+      const unsigned n32 = (unsigned)ns;
+      b0 = P[my_cluster] + r * n32 / k;
+      b1 = P[my_cluster] + (r + 1) * n32 / k;
+    } else {
+      b0 = P[my_cluster] + (long long)r * ns / ksz;
+      b1 = P[my_cluster] + (long long)(r + 1) * ns / ksz;
+    }
     active = b1 > b0;
   }
 
