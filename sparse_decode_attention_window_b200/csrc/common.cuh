@@ -168,6 +168,27 @@ KVC_DEV void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
 }
 KVC_DEV void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
 KVC_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+KVC_DEV uint32_t cluster_nctas() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+// Every thread of every CTA in the cluster: shared-memory writes made before it (release)
+// are visible to every CTA of the cluster after it (acquire).
+KVC_DEV void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+// Loads from another CTA's shared memory (an address from map_to_rank).
+KVC_DEV uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+KVC_DEV unsigned long long ld_cluster_u64(uint32_t addr) {
+  unsigned long long v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 // Bounded wait with cluster-scope acquire (data that other CTAs sent with st.async).
 KVC_DEV bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {

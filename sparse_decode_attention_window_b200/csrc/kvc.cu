@@ -11,6 +11,7 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 
 #include "common.cuh"
 #include "score_simt.cuh"
@@ -123,6 +124,15 @@ bool force_two_pass_score() {
   static const bool v = [] {
     const char* e = getenv("KVC_SCORE_PATH");
     return e && strcmp(e, "twopass") == 0;
+  }();
+  return v;
+}
+
+// KVC_SELECT_PATH=cta keeps selection at one CTA per slot (cross-checks); read once.
+bool force_cta_select() {
+  static const bool v = [] {
+    const char* e = getenv("KVC_SELECT_PATH");
+    return e && strcmp(e, "cta") == 0;
   }();
   return v;
 }
@@ -590,6 +600,93 @@ kvc_status kvc_score(const kvc_shape* shape, const void* q_win, const void* k, c
   return check_launch("kvc_score");
 }
 
+// Selection launch. Few slots: a cluster of k CTAs per slot (select_cluster_kernel), k the
+// largest power of two <= 16 with all S*k CTAs in one wave, at least 128 keys per CTA and
+// each CTA's key range in shared memory; otherwise one CTA per slot (select_kernel).
+int select_cluster_size(int S, int N, int sms, int optin, int* cap_out, size_t* smem_out) {
+  if (force_cta_select()) return 1;
+  for (int k = kvc::SCL_MAX_K; k >= 2; k >>= 1) {
+    if ((long long)S * k > sms) continue;
+    const int per = (N + k - 1) / k;
+    if (per < 128) continue;
+    const int cap = (per + 3) & ~3;
+    const size_t smem = kvc::select_cluster_smem_bytes(cap);
+    if (smem > (size_t)optin) continue;
+    static std::mutex mu;
+    static std::map<std::tuple<int, int, size_t>, int> known;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int n = 0;
+    {
+      std::lock_guard<std::mutex> lk(mu);
+      auto it = known.find({k, dev, smem});
+      if (it != known.end()) {
+        n = it->second;
+      } else {
+        // (set_smem only ever raises the kernel's limit, which launches of other sizes rely on)
+        if (set_smem(kvc::select_cluster_kernel, smem, "kvc_select") != KVC_OK) cudaGetLastError();
+        if (k > 8) cudaFuncSetAttribute(kvc::select_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(k);
+        cfg.blockDim = dim3(kvc::SCL_THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = k;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, kvc::select_cluster_kernel, &cfg) != cudaSuccess) n = 0;
+        cudaGetLastError();
+        known[{k, dev, smem}] = n;
+      }
+    }
+    if (n < S) continue;
+    *cap_out = cap;
+    *smem_out = smem;
+    return k;
+  }
+  return 1;
+}
+
+kvc_status launch_select(kvc::SelectParams p, int S, int N, cudaStream_t stream, const char* what) {
+  DevInfo* di = nullptr;
+  kvc_status rc = dev_info(&di);
+  if (rc != KVC_OK) return rc;
+  int cap = 0;
+  size_t smem = 0;
+  const int k = select_cluster_size(S, N, di->sms, di->smem_optin, &cap, &smem);
+  if (k >= 2) {
+    p.key_cap = cap;
+    if ((rc = set_smem(kvc::select_cluster_kernel, smem, what)) != KVC_OK) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S * k);
+    cfg.blockDim = dim3(kvc::SCL_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = k;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kvc::select_cluster_kernel, p);
+    if (e != cudaSuccess) {
+      cudaGetLastError();                 // not sticky: leave no error for the next check
+      return fail(KVC_ERR_CUDA, "%s: launch: %s", what, cudaGetErrorString(e));
+    }
+  } else {
+    p.key_cap = kvc::select_key_cap(p.L, p.C);
+    smem = kvc::select_smem_bytes(p.key_cap);
+    if ((rc = set_smem(kvc::select_kernel, smem, what)) != KVC_OK) return rc;
+    kvc::select_kernel<<<S, kvc::SEL_THREADS, smem, stream>>>(p);
+  }
+  count_launches(1);
+  return check_launch(what);
+}
+
 kvc_status kvc_select(const kvc_shape* shape, const float* score, const int8_t* policy, const int32_t* budget,
                       float mass, const uint8_t* special_mask, const int32_t* chunk_end, int32_t C, int32_t* idx,
                       int32_t max_sel, int32_t* count, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -618,13 +715,8 @@ kvc_status kvc_select(const kvc_shape* shape, const float* score, const int8_t* 
   p.idx = idx;
   p.max_sel = max_sel;
   p.count = count;
-  p.key_cap = kvc::select_key_cap(shape->L, chunk_end ? C : 0);
   p.n_local = 0;
-  const size_t smem = kvc::select_smem_bytes(p.key_cap);
-  if ((rc = set_smem(kvc::select_kernel, smem, "kvc_select")) != KVC_OK) return rc;
-  kvc::select_kernel<<<shape->n_slots, kvc::SEL_THREADS, smem, stream>>>(p);
-  count_launches(1);
-  return check_launch("kvc_select");
+  return launch_select(p, shape->n_slots, std::max(shape->L, p.C), stream, "kvc_select");
 }
 
 kvc_status kvc_alloc_budgets(const int32_t* counts, int32_t n_layers, int32_t spl, int32_t L, int32_t avg_B,
@@ -865,13 +957,8 @@ kvc_status kvc_select_chunks(const kvc_shape* shape, const float* chunk_score, c
   p.idx = idx;
   p.max_sel = max_sel;
   p.count = count;
-  p.key_cap = kvc::select_key_cap(shape->L, C);
   p.n_local = n_local;
-  const size_t smem = kvc::select_smem_bytes(p.key_cap);
-  if ((rc = set_smem(kvc::select_kernel, smem, "kvc_select_chunks")) != KVC_OK) return rc;
-  kvc::select_kernel<<<shape->n_slots, kvc::SEL_THREADS, smem, stream>>>(p);
-  count_launches(1);
-  return check_launch("kvc_select_chunks");
+  return launch_select(p, shape->n_slots, C, stream, "kvc_select_chunks");
 }
 
 kvc_status kvc_retained_mass(const kvc_shape* shape, const float* score, int32_t N, const int32_t* idx,

@@ -223,6 +223,93 @@ def test_mass_count_closed_forms_on_gpu():
     P.check_mass_count(int(c[2]), _np(sc[2]).astype(np.float64))
 
 
+# slot counts whose selection runs in clusters of 16, 8, 4 and 2 CTAs per slot, and at one CTA per slot
+SELECT_SHAPES = [(1, 4096), (3, 2048), (9, 2048), (18, 1000), (37, 3000), (60, 777), (150, 300)]
+
+
+@pytest.mark.parametrize("S,N", SELECT_SHAPES)
+def test_selection_policies_over_slot_counts(S, N):
+    """kvc_select on given fp32 scores with many ties: top-B (ragged budgets, 0 and >= N
+    included) and the FastGen policies are exact against the oracle; LMBA counts agree
+    within the tie band."""
+    import sparse_decode_attention_window_b200 as kvc
+    g = torch.Generator().manual_seed(7919 * S + N)
+    sc = torch.exp((torch.randn((S, N), generator=g) * 8).round() / 4).float()   # positive, many ties
+    kinds = [kvc.KVC_POL_TOPB, kvc.KVC_POL_MASS_COUNT, kvc.KVC_POL_TOPB, kvc.KVC_POL_LOCAL,
+             kvc.KVC_POL_SPECIAL, kvc.KVC_POL_FULL, kvc.KVC_POL_MASS_COUNT]
+    pol = torch.tensor([kinds[s % len(kinds)] for s in range(S)], dtype=torch.int8)
+    bud = torch.randint(0, N + 4, (S,), generator=g, dtype=torch.int32)
+    bud[0] = N // 3
+    if S > 2:
+        bud[2] = 0
+    if S > 9:
+        bud[9] = N
+    special = (torch.rand((S, N), generator=g) < 0.05).to(torch.uint8)
+    sh = kvc.make_shape(S, 1, 64, N, 1, 1, S, torch.bfloat16)
+    idx = torch.full((S, N), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((S,), -1, dtype=torch.int32, device="cuda")
+    kvc.kvc_select(sh, sc.cuda(), pol.cuda(), bud.cuda(), idx, cnt, mass=0.9, special_mask=special.cuda())
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    idx, cnt = _np(idx), _np(cnt)
+    sc64 = sc.double().numpy()
+    for s in range(S):
+        k = int(pol[s])
+        got = idx[s, :cnt[s]].astype(np.int64)
+        if k == kvc.KVC_POL_TOPB:
+            want = O.top_b(sc64[s], max(int(bud[s]), 0))
+        elif k == kvc.KVC_POL_MASS_COUNT:
+            P.check_mass_count(int(cnt[s]), sc64[s], 0.9, f"slot {s}")
+            continue
+        elif k == kvc.KVC_POL_LOCAL:
+            want = O.local_indices(N, int(bud[s]))
+        elif k == kvc.KVC_POL_SPECIAL:
+            want = O.special_indices(special[s].numpy())
+        else:
+            want = O.full_indices(N)
+        np.testing.assert_array_equal(got, want, err_msg=f"slot {s} policy {k}")
+
+
+@pytest.mark.parametrize("S,C", [(1, 3000), (5, 1200), (9, 2048), (40, 700), (150, 200)])
+@pytest.mark.parametrize("n_local", [0, 3])
+def test_chunk_selection_over_slot_counts(S, C, n_local):
+    """kvc_select_chunks on given fp32 chunk scores with ties and ragged chunk lengths is
+    exact against the oracle for every slot count (cluster sizes 16 down to one CTA)."""
+    import sparse_decode_attention_window_b200 as kvc
+    g = torch.Generator().manual_seed(104729 * S + C + n_local)
+    lens = torch.randint(1, 41, (C,), generator=g)
+    ce = (torch.cumsum(lens, 0) - 1).to(torch.int32)
+    L = int(ce[-1]) + 1
+    sc = torch.exp((torch.randn((S, C), generator=g) * 8).round() / 4).float()
+    tgt = torch.randint(1, L + 4, (S,), generator=g, dtype=torch.int32)
+    tgt[0] = max(1, L // 2)
+    sh = kvc.make_shape(S, 1, 64, L, 1, 1, S, torch.bfloat16)
+    idx = torch.full((S, L), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((S,), -1, dtype=torch.int32, device="cuda")
+    kvc.kvc_select_chunks(sh, sc.cuda(), ce.cuda(), tgt.cuda(), idx, cnt, n_local=n_local)
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    idx, cnt = _np(idx), _np(cnt)
+    for s in range(S):
+        want, _ = O.chunk_select_local(sc[s].double().numpy(), ce.numpy(), int(tgt[s]), n_local)
+        np.testing.assert_array_equal(idx[s, :cnt[s]].astype(np.int64), want, err_msg=f"slot {s}")
+
+
+def test_one_cta_per_slot_selection_on_workloads():
+    """Selection at one CTA per slot (forced here; few slots take thread-block clusters by
+    default) passes the same oracle checks."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, KVC_SELECT_PATH="cta")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                        "-k", "selection_policies_over_slot_counts or chunk_selection_over_slot_counts or "
+                              "llama8b_shape_small_context or zigzag_small or chunk_small or budget_extremes or "
+                              "mass_count_closed_forms or chunk_selection_with_local_chunks"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
 def test_empty_slot_decodes_to_zero_and_append_overflow_is_reported():
     import sparse_decode_attention_window_b200 as kvc
     S, G, d = 3, 2, 64
