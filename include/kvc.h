@@ -12,6 +12,8 @@
  *   kvc_append         one new token per slot per decode step
  *   kvc_decode_attn    split-K GQA decode attention over the ragged packed cache
  *   kvc_append_decode  the two above fused into one launch (the per-step call)
+ *   kvc_append_decode_chain  the same for the loop's later steps, overlapping the
+ *                      previous step's tail
  *
  * Sources: "ZigZagKV: Dynamic KV Cache Compression for Long-context Modeling based
  * on Layer Uncertainty" (arXiv 2412.09036) Eq. 3-7; "Model Tells You What to
@@ -219,6 +221,28 @@ kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const vo
                              const void* q, void* kp, void* vp, const int64_t* off,
                              const int32_t* cap, int32_t* len, int64_t kp_rows, float* out,
                              void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * kvc_append_decode_chain - kvc_append_decode for the steps of a decode loop after its
+ *   first: same arguments and results, plus `stable` [n_slots] int32 (device), a row
+ *   count per slot that the caller guarantees is not written by the kernel issued just
+ *   before this call on `stream`, nor by this call: the kept rows of a compacted cache
+ *   (its count from kvc_select) while the loop only appends. The caller also guarantees
+ *   that this previous kernel writes none of off, cap and stable. The launch then plans
+ *   its work split from cap and starts loading the rows below stable[s] before the
+ *   previous kernel has finished (programmatic dependent launch), which shortens a step
+ *   by the prologue and the first load's latency. The first step after kvc_compact (or
+ *   anything else that rewrites those rows) must use kvc_append_decode. A slot whose
+ *   length turns out below stable[s] breaks the promise: it gets no new token, is
+ *   attended over stable[s] rows, and KVC_DEVERR_INDEX_RANGE is set. stable == NULL:
+ *   KVC_ERR_INVALID_ARG. Other dtypes / G behave
+ *   as kvc_append_decode (the promise is then unused).
+ */
+kvc_status kvc_append_decode_chain(const kvc_shape* shape, const void* k_new, const void* v_new,
+                                   const void* q, void* kp, void* vp, const int64_t* off,
+                                   const int32_t* cap, const int32_t* stable, int32_t* len,
+                                   int64_t kp_rows, float* out, void* ws, size_t ws_bytes,
+                                   cudaStream_t stream);
 
 /*
  * kvc_decode_attn_noalloc - kvc_decode_attn for callers that cannot allocate

@@ -18,7 +18,7 @@ from ._abi import (KvcShape, KvcError, KVC_BF16, KVC_FP32, KVC_POL_TOPB, KVC_POL
 
 __all__ = ["KvcShape", "KvcError", "make_shape", "kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout",
            "kvc_compact", "kvc_append", "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_version",
-           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_select_chunks",
+           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_append_decode_chain", "kvc_select_chunks",
            "kvc_retained_mass", "kvc_profile_heads", "kvc_append_window",
            "library", "KVC_BF16", "KVC_FP32", "KVC_POL_TOPB", "KVC_POL_MASS_COUNT", "KVC_POL_LOCAL",
            "KVC_POL_SPECIAL", "KVC_POL_FULL", "KVC_POL_CHUNK", "KVC_WS_SCORE", "KVC_WS_SELECT", "KVC_WS_DECODE"]
@@ -112,6 +112,16 @@ def kvc_append_decode(shape, k_new, v_new, q, kp, vp, off, cap, length, out, ws,
            library().kvc_append_decode(ctypes.byref(shape), _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(kp), _ptr(vp),
                                        _ptr(off), _ptr(cap), _ptr(length), int(kp.shape[0]), _ptr(out), _ptr(ws),
                                        ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def kvc_append_decode_chain(shape, k_new, v_new, q, kp, vp, off, cap, stable, length, out, ws, stream=None):
+    """kvc_append_decode for a decode-loop step after the first: `stable` holds per slot
+    a row count that the previous kernel on the stream does not write (see include/kvc.h)."""
+    _check("kvc_append_decode_chain",
+           library().kvc_append_decode_chain(ctypes.byref(shape), _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(kp),
+                                             _ptr(vp), _ptr(off), _ptr(cap), _ptr(stable), _ptr(length),
+                                             int(kp.shape[0]), _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                             _stream(stream)))
 
 
 def kvc_decode_attn_noalloc(shape, q, kp, vp, off, length, out, stream=None):

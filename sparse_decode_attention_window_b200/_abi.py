@@ -22,7 +22,7 @@ KVC_WS_SCORE, KVC_WS_SELECT, KVC_WS_DECODE = 0, 1, 2
 EXPORTS = ["kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout", "kvc_compact", "kvc_append",
            "kvc_append_window",
            "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_last_error", "kvc_version",
-           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_select_chunks",
+           "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_append_decode_chain", "kvc_select_chunks",
            "kvc_retained_mass", "kvc_profile_heads"]
 
 
@@ -69,6 +69,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "kvc_launch_count": (ctypes.c_ulonglong, []),
         "kvc_decode_attn_noalloc": (i32, [sh, vp, vp, vp, vp, vp, i64, vp, vp]),
         "kvc_append_decode": (i32, [sh, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
+        "kvc_append_decode_chain": (i32, [sh, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp]),
         "kvc_select_chunks": (i32, [sh, vp, vp, i32, vp, i32, vp, i32, vp, vp]),
         "kvc_retained_mass": (i32, [sh, vp, i32, vp, i32, vp, vp, vp]),
         "kvc_profile_heads": (i32, [sh, vp, vp, i32, f32, vp, vp, vp]),

@@ -121,6 +121,11 @@ struct DecodeParams {
   const void* v_new;
   const int32_t* cap;
   int32_t* len_out;  // = len; incremented by the last CTA to finish
+  // optional (fused append, tensor-core kernel): rows [0, stable[s]) of slot s are written
+  // neither by the previous kernel on the stream nor by this launch, and off, cap, stable
+  // are not written by the previous kernel either; the launch may then plan and load those
+  // rows before the previous kernel has finished
+  const int32_t* stable;
 };
 
 // The last CTA to finish slot s merges the slot's partials (CTAs cfirst..clast, stored

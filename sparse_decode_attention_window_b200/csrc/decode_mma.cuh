@@ -49,10 +49,11 @@ constexpr float DM_LAZY_LOG2 = 8.f;
 constexpr int DM_MIN_TOKENS_PER_CTA = 64;            // token split: no CTA gets less than a tile
 constexpr long long DM_SEG_COST = 128;               // token split: fixed work of one slot segment, in tokens
 constexpr int DM_MAX_CLUSTER = 8;
+constexpr int DM_APPENDS = 1 << 30;                  // flag in the per-slot row count: the last row is appended
 
 // Shared-memory layout of decode_mma_kernel (host and device agree on it).
 struct DmLayout {
-  size_t stages, qbuf, bars, P, offs, wm, wo, xr, app, total;
+  size_t stages, qbuf, bars, P, offs, wm, wo, xr, vl, total;
   template <int D>
   KVC_HD static DmLayout make(int S, int G, int grid, int nst) {
     using C = DmCfg<D>;
@@ -62,13 +63,13 @@ struct DmLayout {
     l.qbuf = o;    o += (size_t)nst * G * D * 2;                     // the slot's q, one per stage
     l.bars = o;    o += (2 * C::MAX_STAGES + 1) * sizeof(uint64_t);  // full, empty, rank 0's record barrier
     l.P = o;       o += (size_t)(S + 1) * sizeof(long long);
-    l.offs = o;    o += (size_t)S * sizeof(long long);
+    l.offs = o;    o += (size_t)S * sizeof(int);                      // row offsets (< 2^31, as TMA rows)
     l.wm = o;      o += 2 * C::CONS_WARPS * 8 * sizeof(float);       // per-warp max and sum, 8 heads
     l.wo = o;      o += (size_t)C::CONS_WARPS * G * C::WO_STRIDE * sizeof(float);
     // per-slot clusters: the k CTA records [k][G*D + 2G, padded] that rank 0 merges
     const size_t clu = 2 * S <= grid ? (size_t)DM_MAX_CLUSTER * partial_stride(G, D) * sizeof(float) : 0;
     l.xr = o;      o += clu;
-    l.app = o;     o += (size_t)S;
+    l.vl = o;      o += (size_t)S * sizeof(int);                      // rows attended per slot | DM_APPENDS
     l.total = o + 1024 + 16;                                          // base alignment slack
     return l;
   }
@@ -208,19 +209,21 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   uint64_t* empty = full + C::MAX_STAGES;
   uint64_t* rec_bar = empty + C::MAX_STAGES;   // rank 0 of a slot cluster: the other CTAs' records (st.async bytes)
   long long* P = reinterpret_cast<long long*>(sm + lay.P);
-  long long* offs = reinterpret_cast<long long*>(sm + lay.offs);
+  int* offs = reinterpret_cast<int*>(sm + lay.offs);
   float* wm = reinterpret_cast<float*>(sm + lay.wm);        // [warp][8] maxima
   float* wl = wm + C::CONS_WARPS * 8;                        // [warp][8] sums
   float* wo = reinterpret_cast<float*>(sm + lay.wo);        // [warp][G][WO_STRIDE]
   float* xr = reinterpret_cast<float*>(sm + lay.xr);
-  unsigned char* app = sm + lay.app;
+  int* vlen_sh = reinterpret_cast<int*>(sm + lay.vl);
+  // rows attended in slot s; with the fused append the last of them is the new token
+  auto vlen = [&](int s) { return vlen_sh[s] & ~DM_APPENDS; };
+  auto appends = [&](int s) { return (vlen_sh[s] & DM_APPENDS) != 0; };
   __shared__ unsigned long long scan_sh[33];
   __shared__ int last_flag;
   __shared__ int abort_flag;
   __shared__ unsigned long long max_len_sh;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // Nothing before the dependency wait reads global memory that an earlier kernel writes.
   if (tid == 0) {
     max_len_sh = 0;
     abort_flag = 0;
@@ -241,39 +244,81 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   // any CTA sends to another (the matching wait comes before the first st.async)
   if (ksz >= 2) cluster_arrive_relaxed();
   bool cl_waited = false;
-  // Launched with programmatic stream serialization: wait until the previous kernel on
-  // the stream has completed and its writes are visible, then let the next one launch.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // The work is planned on the slots' capacities when the call appends (the decode loop
+  // never writes cap), otherwise on the lengths. `early`: the caller promises that the
+  // previous kernel on the stream wrote none of off, cap, stable and no K/V row below
+  // stable[s]; the plan, and the loads of the first tiles below stable[s], then run before
+  // the dependency wait (programmatic dependent launch). Otherwise nothing before the wait
+  // reads global memory that an earlier kernel writes.
+  const bool plan_cap = a.append != 0;
+  const bool early = plan_cap && a.stable != nullptr;
+  if (!early) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
 
-  // One slot's length (clipped to the buffer); with the fused append, a slot that has
-  // room gets its new token as its last row.
-  auto slot_len = [&](int s, unsigned char* ap_out, bool flag_overflow) -> long long {
-    const int ln = a.len[s];
-    const long long os = a.off[s];
-    const int cp = a.append ? a.cap[s] : 0;
-    long long n = max(ln, 0);
-    offs[s] = os;
-    const long long room = a.kp_rows - os;
-    if (n > room) { kvc_flag(KVC_DEVERR_INDEX_RANGE); n = room > 0 ? room : 0; }
-    unsigned char ap = 0;
-    if (a.append) {
-      if (ln >= 0 && n < cp && n < room) { ap = 1; ++n; }
-      else if (flag_overflow) kvc_flag(KVC_DEVERR_APPEND_OVERFLOW);
+  // Fused append, slot s of plan length n: the rows attended (*vl) and whether the new
+  // token is the last of them (*ap) - the slot has room below cap and the buffer. The same
+  // test decides, in the CTA that ends last, which lengths grow.
+  auto append_rows = [&](int s, int ln, int cp, long long n, long long* vl_out, bool* ap_out) {
+    const long long room = a.kp_rows - offs[s];
+    long long vl = max(ln, 0);
+    bool bad = false;
+    if (vl > room) {
+      bad = true;
+      vl = room > 0 ? room : 0;
     }
+    bool ap = ln >= 0 && vl < cp && vl < room && vl < n;
+    if (ap) ++vl;
+    if (vl > n) {                      // a length beyond the capacity
+      bad = true;
+      vl = n;
+    }
+    if (early) {
+      const long long st = min((long long)max(a.stable[s], 0), n);
+      if (vl < st) {
+        bad = true;
+        ap = false;
+        vl = st;
+      }
+    }
+    *vl_out = vl;
     *ap_out = ap;
-    return n;
+    return bad;
   };
-  // prefix of the lengths over all slots, and the largest one
+  // plan lengths (clipped to the buffer), their prefix over the slots, and the largest one
   unsigned long long carry = 0, mxl = 0;
   for (int base = 0; base < S; base += blockDim.x) {
     const int s = base + tid;
     unsigned long long x = 0;
     if (s < S) {
-      unsigned char ap;
-      x = (unsigned long long)slot_len(s, &ap, blockIdx.x == 0);
-      app[s] = ap;
+      // every global read of the slot first, so that their latencies overlap
+      long long os = a.off[s];
+      const int cp = plan_cap ? a.cap[s] : 0;   // cap is NULL for a plain decode
+      const int ln = (!plan_cap || !early) ? a.len[s] : 0;
+      if (os < 0 || os > a.kp_rows) {   // an offset outside the buffer: nothing of the slot is read or written
+        kvc_flag(KVC_DEVERR_INDEX_RANGE);
+        os = a.kp_rows;
+      }
+      offs[s] = (int)os;                // kp_rows < 2^31 (checked at launch)
+      const long long room = a.kp_rows - os;
+      long long n = max(plan_cap ? cp : ln, 0);
+      if (n > room) {
+        if (!plan_cap) kvc_flag(KVC_DEVERR_INDEX_RANGE);
+        n = room > 0 ? room : 0;
+      }
+      x = (unsigned long long)n;
       mxl = x > mxl ? x : mxl;
+      if (!early) {                     // the lengths are readable already: rows attended, in the same pass
+        int v = (int)n;
+        if (plan_cap) {
+          long long vl;
+          bool ap;
+          append_rows(s, ln, cp, n, &vl, &ap);
+          v = (int)vl | (ap ? DM_APPENDS : 0);
+        }
+        vlen_sh[s] = v;
+      }
     }
     unsigned long long tot;
     const unsigned long long before = carry + block_exclusive_scan<unsigned long long>(x, scan_sh, &tot);
@@ -288,13 +333,6 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   if (lane == 0) atomicMax(&max_len_sh, mxl);
   if (tid == 0) P[S] = (long long)carry;
   __syncthreads();
-
-  // Fused append: every CTA has read len once it gets here. Its ticket is taken now but
-  // only looked at when the CTA ends; the CTA that drew the last ticket then publishes
-  // the new lengths (nothing in this launch reads len after its prologue).
-  int ticket = -1;
-  if (a.append && tid == 0)
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(&a.counters[S]), "r"(1) : "memory");
 
   const long long N = P[S];
   const int nC = gridDim.x, c = blockIdx.x;
@@ -313,7 +351,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
     return max(P[lo], x - (long long)(lo + 1) * DM_SEG_COST);
   };
   // per-slot clusters: launched in clusters, every slot has one, they fill >= 3/4 of
-  // the grid, and the lengths are near uniform (the same test in every CTA)
+  // the grid, and the plan lengths are near uniform (the same test in every CTA)
   const bool per_slot = ksz >= 2 && (long long)S * ksz <= nC && 4LL * S * ksz >= 3LL * nC &&
                         4LL * (long long)max_len_sh * S <= 5LL * N;
   const int my_cluster = per_slot ? (int)((unsigned)c / (unsigned)ksz) : c;
@@ -361,6 +399,92 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   };
   const uint32_t q_bytes = (uint32_t)(G * D * 2);
 
+  // Early: the producer starts the K/V loads of the first full tiles of the CTA's first
+  // segment that lie below stable[s] - the same tiles, in the same order and stages, that
+  // its main loop takes first. They carry no q: the consumers read the first segment's q
+  // themselves after the wait.
+  int nspec = 0;
+  if (early && warp == C::CONS_WARPS && lane == 0 && active) {
+    const int s = slot_of(b0);
+    const long long seg_end = min(b1, P[s + 1]);
+    const long long st_end = min(seg_end, P[s] + (long long)max(a.stable[s], 0));
+    for (long long u = b0; u + C::TILE <= st_end && nspec < nst; u += C::TILE) {
+      const int row0 = (int)(offs[s] + (u - P[s]));
+      unsigned char* kdst = stages + nspec * C::STAGE_BYTES;
+      unsigned char* vdst = kdst + C::KB * C::REGION;
+      mbar_arrive_expect_tx(&full[nspec], 2 * C::KB * C::REGION);
+#pragma unroll
+      for (int kb = 0; kb < C::KB; ++kb) {
+        tma_load_2d(kdst + kb * C::REGION, &mk64, kb * 64, row0, &full[nspec]);
+        tma_load_2d(vdst + kb * C::REGION, &mv64, kb * 64, row0, &full[nspec]);
+      }
+      ++nspec;
+    }
+  }
+  if (early) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
+  // Early: the consumers' Q^T operand of the first segment, straight from global memory
+  // (q is written by the previous kernel; its tiles carry none), overlapping the reads below
+  const int g_ = (tid & 31) >> 2, qd_ = tid & 3;
+  const int qhead0 = PACK ? (g_ & 3) : g_;
+  uint32_t q0[C::KSTEPS][2];
+  if (early && warp < C::CONS_WARPS && active) {
+    const unsigned char* qg = static_cast<const unsigned char*>(a.q) + (size_t)slot_of(b0) * q_bytes;
+#pragma unroll
+    for (int ks = 0; ks < C::KSTEPS; ++ks) {
+      uint32_t v0 = 0, v1 = 0;
+      if (qhead0 < G) {
+        const unsigned char* qr = qg + ((size_t)qhead0 * D + ks * 16 + 2 * qd_) * 2;
+        v0 = __ldg(reinterpret_cast<const unsigned int*>(qr));
+        v1 = __ldg(reinterpret_cast<const unsigned int*>(qr + 16));
+      }
+      q0[ks][0] = v0;
+      q0[ks][1] = v1;
+    }
+  }
+
+  // Early: rows attended in each slot this CTA touches, now that the lengths (written by
+  // the previous launch) can be read: the length plus the new token as the last row where
+  // the slot has room. A slot is never attended over fewer than its stable rows; a shorter
+  // length breaks the caller's promise: flagged, and the slot gets no new token.
+  // The producer, maybe still issuing those loads, takes no part: the consumers read the
+  // lengths, sync among themselves and release the producer through barrier 2.
+  if (early && warp < C::CONS_WARPS) {
+    int s_lo = 0, s_hi = -1;
+    if (per_slot) {
+      if (in_slot_cluster) s_lo = s_hi = my_cluster;
+    } else if (active) {
+      s_lo = slot_of(b0);
+      s_hi = slot_of(b1 - 1);
+    }
+    for (int s = s_lo + tid; s <= s_hi; s += C::CONS_THREADS) {
+      const long long n = P[s + 1] - P[s];
+      int v = (int)n;
+      if (plan_cap) {
+        long long vl;
+        bool ap;
+        append_rows(s, a.len[s], a.cap[s], n, &vl, &ap);
+        v = (int)vl | (ap ? DM_APPENDS : 0);
+      }
+      vlen_sh[s] = v;
+    }
+    named_bar_sync(3, C::CONS_THREADS);
+    named_bar_arrive(2, C::THREADS);
+  } else if (early) {
+    __syncwarp();
+    named_bar_sync(2, C::THREADS);     // the consumers have written the rows attended
+  }
+
+  // Fused append: every CTA has read len once it gets here. Its ticket is taken now (a
+  // release: the CTA's reads of len come first; no acquire, so warp 0 does not wait for
+  // it) but only looked at when the CTA ends; the CTA that drew the last ticket then
+  // publishes the new lengths (nothing in this launch reads len after this point).
+  int ticket = -1;
+  if (a.append && tid == 0)
+    asm volatile("atom.release.gpu.global.add.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(&a.counters[S]), "r"(1) : "memory");
+
   if (warp == C::CONS_WARPS) {
     // ---------------- producer: TMA of 64-token K and V tiles (16-row boxes for a partial
     // tile); the first tile of a segment also brings the slot's q
@@ -372,8 +496,14 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       for (long long t = b0; t < b1 && ok;) {
         const int s = slot_of(t);
         const long long seg_end = min(b1, P[s + 1]);
-        for (long long u = t; u < seg_end; u += C::TILE) {
-          const int rows = (int)min((long long)C::TILE, seg_end - u);
+        const long long vend = min(seg_end, P[s] + (long long)vlen(s));   // attended rows of the segment
+        for (long long u = t; u < vend; u += C::TILE) {
+          const int rows = (int)min((long long)C::TILE, vend - u);
+          if (issued < nspec) {            // on its way since before the wait
+            ++issued;
+            if (++stage == nst) { stage = 0; ph ^= 1; }
+            continue;
+          }
           // the first nst tiles find their stages free
           if ((issued >= nst && !mbar_wait(&empty[stage], ph ^ 1)) || *(volatile int*)&abort_flag) {
             ok = false;
@@ -438,6 +568,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       pending_empty = false;
       const int s = slot_of(t);
       const long long seg_end = active ? min(b1, P[s + 1]) : t;
+      const long long vend = min(seg_end, P[s] + (long long)vlen(s));   // attended rows of the segment
 
       uint32_t qb[C::KSTEPS][2];
       float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
@@ -446,16 +577,24 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       for (int dt = 0; dt < C::DTILES; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
 
       bool have_q = false;
-      for (long long u = t; u < seg_end; u += C::TILE, ++tile_k) {
+      for (long long u = t; u < vend; u += C::TILE, ++tile_k) {
         if ((int)(tile_k & 1) != grp) {      // the other group's tile
           if (++stage == nst) { stage = 0; ph ^= 1; }
           continue;
         }
-        const int rows = (int)min((long long)C::TILE, seg_end - u);
+        const int rows = (int)min((long long)C::TILE, vend - u);
         if (!mbar_wait(&full[stage], ph)) {   // the group's warps wait on this barrier: all stop here
           *(volatile int*)&abort_flag = 1;
           aborted = true;
           break;
+        }
+        if (!have_q && early && t == b0) {   // the first segment's q, read after the wait
+          have_q = true;
+#pragma unroll
+          for (int ks = 0; ks < C::KSTEPS; ++ks) {
+            qb[ks][0] = q0[ks][0];
+            qb[ks][1] = q0[ks][1];
+          }
         }
         if (!have_q) {
           have_q = true;
@@ -479,12 +618,13 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         // fused append: the slot's new token is its last valid row; if it falls in this
         // warp's m-tile, put it into the staged tile (the cache row is stale) and the cache
         bool patched = false;
-        if (app[s] && P[s + 1] - 1 >= u && P[s + 1] - 1 < u + rows) {
-          const int tr = (int)(P[s + 1] - 1 - u);
+        const long long arow_t = appends(s) ? P[s] + vlen(s) - 1 : -1;   // the appended token, in plan space
+        if (arow_t >= u && arow_t < u + rows) {
+          const int tr = (int)(arow_t - u);
           if (tr >= mrow0 && tr < mrow0 + 16) {
             const uint4* kn = static_cast<const uint4*>(a.k_new) + (size_t)s * (D / 8);
             const uint4* vn = static_cast<const uint4*>(a.v_new) + (size_t)s * (D / 8);
-            const size_t dst_row = (size_t)(offs[s] + (P[s + 1] - 1 - P[s])) * (D / 8);
+            const size_t dst_row = (size_t)(offs[s] + vlen(s) - 1) * (D / 8);
             for (int ch = lane; ch < D / 8; ch += 32) {
               const uint4 kv = kn[ch], vv = vn[ch];
               *reinterpret_cast<uint4*>(Ks + (ch >> 3) * C::REGION + swz(tr, ch & 7)) = kv;
@@ -715,26 +855,20 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       const int rs = partial_stride(G, D);
       if (tid == 0) mbar_arrive_expect_tx(rec_bar, (uint32_t)((ksz - 1) * (G * D + 2 * G) * 4));
       if (mbar_wait_cluster(rec_bar, 0)) {
-        float* sc = wo;              // [ksz][8] weights, then 1 / sum [8] (the combine buffer is free)
-        float* linv = sc + 8 * 8;
-        if (tid < G) {
-          float M = -INFINITY;
-          for (int r = 0; r < ksz; ++r) M = fmaxf(M, xr[r * rs + G * D + tid]);
-          float Lt = 0.f;
-          for (int r = 0; r < ksz; ++r) {
-            const float mr = xr[r * rs + G * D + tid];
-            const float w = mr == -INFINITY ? 0.f : ex2_ftz(mr - M);
-            sc[r * 8 + tid] = w;
-            Lt += xr[r * rs + G * D + G + tid] * w;
-          }
-          linv[tid] = Lt > 0.f ? 1.f / Lt : 0.f;
-        }
-        named_bar_sync(1, C::CONS_THREADS);
+        // each thread weighs the records for its own outputs' head (no barrier)
         for (int e = tid; e < G * D; e += C::CONS_THREADS) {
           const int h = e / D;
-          float acc = 0.f;
-          for (int r = 0; r < ksz; ++r) acc += sc[r * 8 + h] * xr[r * rs + e];
-          a.out[(size_t)my_cluster * G * D + e] = acc * linv[h];
+          float M = -INFINITY;
+          for (int r = 0; r < ksz; ++r) M = fmaxf(M, xr[r * rs + G * D + h]);
+          float acc = 0.f, Lt = 0.f;
+          for (int r = 0; r < ksz; ++r) {
+            const float mr = xr[r * rs + G * D + h];
+            const float w = mr == -INFINITY ? 0.f : ex2_ftz(mr - M);
+            Lt += xr[r * rs + G * D + G + h] * w;
+            acc += w * xr[r * rs + e];
+          }
+          const float linv = Lt > 0.f ? 1.f / Lt : 0.f;
+          a.out[(size_t)my_cluster * G * D + e] = acc * linv;
         }
       }
     }
@@ -743,11 +877,20 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   if (ksz >= 2 && !cl_waited) cluster_wait();
 
   if (a.append) {
-    if (tid == 0) last_flag = ticket == (int)gridDim.x - 1;
+    if (tid == 0) {
+      last_flag = ticket == (int)gridDim.x - 1;
+      if (last_flag) asm volatile("fence.acq_rel.gpu;" ::: "memory");   // after every CTA's reads of len
+    }
     __syncthreads();
     if (last_flag) {
-      for (int s = tid; s < S; s += blockDim.x)
-        if (app[s]) a.len_out[s] = a.len[s] + 1;
+      // the same test as the rows pass above, for every slot
+      for (int s = tid; s < S; s += blockDim.x) {
+        long long vl;
+        bool ap;
+        if (append_rows(s, a.len[s], a.cap[s], P[s + 1] - P[s], &vl, &ap)) kvc_flag(KVC_DEVERR_INDEX_RANGE);
+        if (ap) a.len_out[s] = a.len[s] + 1;
+        else kvc_flag(KVC_DEVERR_APPEND_OVERFLOW);
+      }
       if (tid == 0) a.counters[S] = 0;
     }
   }

@@ -280,6 +280,8 @@ kvc_status launch_decode_mma(const kvc::DecodeParams& p, int G, int sms, cudaStr
   // use it). The grid is the resident clusters, at most SMs / k of them; a size is kept
   // only when the slot-count half of the kernel's test can pass (S k <= grid <= 4/3 S k),
   // otherwise the launch is a plain one CTA per SM.
+  if (p.kp_rows > INT32_MAX)   // TMA row coordinates are 32-bit
+    return fail(KVC_ERR_UNSUPPORTED, "kvc_decode_attn: %lld cache rows (> 2^31 - 1)", (long long)p.kp_rows);
   int k = p.S > 0 ? sms / p.S : 0;
   if (k > DM_MAX_CLUSTER) k = DM_MAX_CLUSTER;
   if (!allow_cluster || force_token_split()) k = 1;
@@ -891,28 +893,30 @@ kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const 
   return launch_decode_any(shape, p, di->sms, stream, /*allow_cluster=*/false);
 }
 
-kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const void* v_new, const void* q, void* kp,
-                             void* vp, const int64_t* off, const int32_t* cap, int32_t* len, int64_t kp_rows,
-                             float* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+namespace {
+kvc_status append_decode(const char* what, const kvc_shape* shape, const void* k_new, const void* v_new,
+                         const void* q, void* kp, void* vp, const int64_t* off, const int32_t* cap,
+                         const int32_t* stable, int32_t* len, int64_t kp_rows, float* out, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
   kvc_status rc = check_shape(shape, false);
   if (rc != KVC_OK) return rc;
   if (!k_new || !v_new || !q || !kp || !vp || !off || !cap || !len || !out)
-    return fail(KVC_ERR_INVALID_ARG, "kvc_append_decode: NULL pointer argument");
+    return fail(KVC_ERR_INVALID_ARG, "%s: NULL pointer argument", what);
   if (shape->dtype != KVC_BF16 || shape->G > 8 || force_simt_decode()) {
     // the CUDA-core decode has no fused append: the two calls in sequence
     if ((rc = kvc_append(shape, k_new, v_new, off, cap, len, kp, vp, kp_rows, stream)) != KVC_OK) return rc;
     return kvc_decode_attn(shape, q, kp, vp, off, len, kp_rows, out, ws, ws_bytes, stream);
   }
   if (shape->n_slots > kvc::DEC_MAX_SLOTS)
-    return fail(KVC_ERR_UNSUPPORTED, "kvc_append_decode: %d slots > %d", shape->n_slots, kvc::DEC_MAX_SLOTS);
+    return fail(KVC_ERR_UNSUPPORTED, "%s: %d slots > %d", what, shape->n_slots, kvc::DEC_MAX_SLOTS);
   if (!aligned16(q) || !aligned16(kp) || !aligned16(vp) || !aligned16(ws) || !aligned16(k_new) || !aligned16(v_new) ||
       !aligned16(out))
-    return fail(KVC_ERR_INVALID_ARG, "kvc_append_decode: buffers must be 16-byte aligned");
+    return fail(KVC_ERR_INVALID_ARG, "%s: buffers must be 16-byte aligned", what);
   DevInfo* di = nullptr;
   if ((rc = dev_info(&di)) != KVC_OK) return rc;
   const DecodeWs w = decode_ws_layout(shape, di->sms);
   if (!ws || ws_bytes < w.total)
-    return fail(KVC_ERR_WORKSPACE, "kvc_append_decode: workspace %zu B < required %zu B", ws_bytes, w.total);
+    return fail(KVC_ERR_WORKSPACE, "%s: workspace %zu B < required %zu B", what, ws_bytes, w.total);
   unsigned char* wsb = static_cast<unsigned char*>(ws);
   kvc::DecodeParams p{};
   p.q = q;
@@ -931,7 +935,25 @@ kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const vo
   p.v_new = v_new;
   p.cap = cap;
   p.len_out = len;
+  p.stable = stable;
   return launch_decode_any(shape, p, di->sms, stream);
+}
+}  // namespace
+
+kvc_status kvc_append_decode(const kvc_shape* shape, const void* k_new, const void* v_new, const void* q, void* kp,
+                             void* vp, const int64_t* off, const int32_t* cap, int32_t* len, int64_t kp_rows,
+                             float* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return append_decode("kvc_append_decode", shape, k_new, v_new, q, kp, vp, off, cap, nullptr, len, kp_rows, out, ws,
+                       ws_bytes, stream);
+}
+
+kvc_status kvc_append_decode_chain(const kvc_shape* shape, const void* k_new, const void* v_new, const void* q,
+                                   void* kp, void* vp, const int64_t* off, const int32_t* cap, const int32_t* stable,
+                                   int32_t* len, int64_t kp_rows, float* out, void* ws, size_t ws_bytes,
+                                   cudaStream_t stream) {
+  if (!stable) return fail(KVC_ERR_INVALID_ARG, "kvc_append_decode_chain: stable is NULL");
+  return append_decode("kvc_append_decode_chain", shape, k_new, v_new, q, kp, vp, off, cap, stable, len, kp_rows, out,
+                       ws, ws_bytes, stream);
 }
 
 kvc_status kvc_select_chunks(const kvc_shape* shape, const float* chunk_score, const int32_t* chunk_end, int32_t C,

@@ -16,7 +16,7 @@ import torch
 import math
 
 from . import (kvc_score, kvc_select, kvc_alloc_budgets, kvc_layout, kvc_compact, kvc_append, kvc_decode_attn,
-               kvc_append_decode, kvc_select_chunks, kvc_append_window, KVC_POL_LOCAL,
+               kvc_append_decode, kvc_append_decode_chain, kvc_select_chunks, kvc_append_window, KVC_POL_LOCAL,
                kvc_workspace_size, make_shape, KVC_WS_SCORE, KVC_WS_DECODE, KVC_POL_TOPB, KVC_POL_MASS_COUNT,
                KVC_POL_CHUNK)
 
@@ -36,6 +36,7 @@ class KvcPipeline:
     def __init__(self, wl, inp, device=None, decode_boundaries=None):
         self.wl = wl
         self.inp = inp
+        self._chained = False              # True while the last kernel issued was a decode step's
         dev = torch.device(device) if device is not None else inp.k.device
         self.dev = dev
         S, G, d, L = wl.n_slots, wl.G, wl.d, wl.L
@@ -160,6 +161,7 @@ class KvcPipeline:
         kvc_layout(self.count, self.wl.reserve, self.off, self.cap, stream=stream)
         kvc_compact(self.shape, self.inp.k, self.inp.v, self.idx, self.count, self.off, self.kp, self.vp, self.len,
                     stream=stream)
+        self._chained = False              # the next decode follows a kernel that wrote the kept rows
 
     def compress(self, stream=None):
         self.score_step(stream)
@@ -182,9 +184,15 @@ class KvcPipeline:
             kvc_append_window(self.shape, k_new, v_new, self.off, self.cap, self.len, self.window, self.head,
                               self.kp, self.vp, stream=stream)
             kvc_decode_attn(self.shape, q, self.kp, self.vp, self.off, self.len, out, self.ws_decode, stream=stream)
+        elif fused and self._chained:
+            # the previous step's launch wrote only its appended rows: the kept rows
+            # [0, count) may be loaded before it ends
+            kvc_append_decode_chain(self.shape, k_new, v_new, q, self.kp, self.vp, self.off, self.cap, self.count,
+                                    self.len, out, self.ws_decode, stream=stream)
         elif fused:
             kvc_append_decode(self.shape, k_new, v_new, q, self.kp, self.vp, self.off, self.cap, self.len, out,
                               self.ws_decode, stream=stream)
+            self._chained = True
         else:
             kvc_append(self.shape, k_new, v_new, self.off, self.cap, self.len, self.kp, self.vp, stream=stream)
             kvc_decode_attn(self.shape, q, self.kp, self.vp, self.off, self.len, out, self.ws_decode, stream=stream)
@@ -211,6 +219,7 @@ class KvcPipeline:
         kvc_layout(self.count, wl.steps - t - 1, self.off, self.cap, stream=stream)
         kvc_compact(self.shape_full, self.kf, self.vf, self.idx, self.count, self.off, self.kp, self.vp, self.len,
                     stream=stream)
+        self._chained = False
 
     def run(self, steps=None, record=False, stream=None):
         self.compress(stream)

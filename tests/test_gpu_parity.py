@@ -494,6 +494,86 @@ def test_fused_append_decode_overflow_keeps_old_rows():
     kvc.kvc_get_status()
 
 
+@pytest.mark.parametrize("S,counts", [(32, None), (5, [1000, 3, 0, 64, 700]), (70, None)])
+def test_chained_append_decode_is_bit_identical(S, counts):
+    """kvc_append_decode_chain (the kept rows may load before the previous launch ends)
+    returns bit for bit what kvc_append_decode returns, step after step, on uniform,
+    ragged and many-slot caches; the results match the oracle."""
+    import sparse_decode_attention_window_b200 as kvc
+    G, d, steps = 4, 128, 12
+    g = torch.Generator().manual_seed(S)
+    cnt = (torch.full((S,), 1024, dtype=torch.int32) if counts is None and S <= 32 else
+           torch.randint(0, 900, (S,), generator=g, dtype=torch.int32) if counts is None else
+           torch.tensor(counts, dtype=torch.int32))
+    sh = kvc.make_shape(S, G, d, int(cnt.max()) + steps, 0, S, 1, torch.bfloat16)
+    count = cnt.cuda()
+    off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    cap = torch.empty(S, dtype=torch.int32, device="cuda")
+    kvc.kvc_layout(count, steps, off, cap)
+    rows = int(off[-1])
+    kp = torch.randn(rows, d, generator=g).to(torch.bfloat16).cuda()
+    vp = torch.randn(rows, d, generator=g).to(torch.bfloat16).cuda()
+    kp0, vp0 = kp.clone(), vp.clone()
+    q = torch.randn(steps, S * G, d, generator=g).to(torch.bfloat16).cuda()
+    kn = torch.randn(steps, S, d, generator=g).to(torch.bfloat16).cuda()
+    vn = torch.randn(steps, S, d, generator=g).to(torch.bfloat16).cuda()
+    ws = torch.zeros(kvc.kvc_workspace_size(kvc.KVC_WS_DECODE, sh), dtype=torch.uint8, device="cuda")
+    outs = {}
+    for chained in (False, True):
+        kp.copy_(kp0)
+        vp.copy_(vp0)
+        ln = count.clone()
+        o = torch.empty((steps, S * G, d), device="cuda")
+        for t in range(steps):
+            if chained and t > 0:
+                kvc.kvc_append_decode_chain(sh, kn[t], vn[t], q[t], kp, vp, off, cap, count, ln, o[t], ws)
+            else:
+                kvc.kvc_append_decode(sh, kn[t], vn[t], q[t], kp, vp, off, cap, ln, o[t], ws)
+        torch.cuda.synchronize()
+        kvc.kvc_get_status()
+        assert torch.equal(ln, count + steps)
+        outs[chained] = _np(o)
+    np.testing.assert_array_equal(outs[True], outs[False])
+    offs = _np(off)
+    for s in sorted({0, S // 2, S - 1}):
+        c = int(cnt[s])
+        keys = torch.cat([kp0[offs[s]:offs[s] + c], kn[:, s]]).cpu()
+        vals = torch.cat([vp0[offs[s]:offs[s] + c], vn[:, s]]).cpu()
+        for t in (0, steps - 1):
+            n = c + t + 1
+            ref = O.decode_attention(q[t, s * G:(s + 1) * G].cpu(), keys[:n], vals[:n], [0, n], [n], G)
+            P.check_out(outs[True][t, s * G:(s + 1) * G], ref, "bf16", f"slot {s} step {t}")
+
+
+def test_chained_append_decode_reports_a_broken_promise():
+    """stable[s] above a slot's length is flagged; that slot gets no new token and the
+    launch writes nothing outside the slots."""
+    import sparse_decode_attention_window_b200 as kvc
+    S, G, d = 4, 4, 128
+    sh = kvc.make_shape(S, G, d, 512, 0, S, 1, torch.bfloat16)
+    count = torch.tensor([300, 200, 64, 0], dtype=torch.int32, device="cuda")
+    off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    cap = torch.empty(S, dtype=torch.int32, device="cuda")
+    kvc.kvc_layout(count, 4, off, cap)
+    rows = int(off[-1])
+    kp = torch.randn(rows, d, device="cuda").to(torch.bfloat16)
+    vp = torch.randn(rows, d, device="cuda").to(torch.bfloat16)
+    q = torch.randn(S * G, d, device="cuda").to(torch.bfloat16)
+    kn = torch.randn(S, d, device="cuda").to(torch.bfloat16)
+    out = torch.empty((S * G, d), device="cuda")
+    ws = torch.zeros(kvc.kvc_workspace_size(kvc.KVC_WS_DECODE, sh), dtype=torch.uint8, device="cuda")
+    ln = count.clone()
+    stable = count.clone()
+    stable[1] = 260                    # above slot 1's length (and capacity)
+    kvc.kvc_append_decode_chain(sh, kn, kn, q, kp, vp, off, cap, stable, ln, out, ws)
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.kvc_get_status()
+    assert "index-out-of-range" in str(e.value) and "wait-timeout" not in str(e.value)
+    assert ln.cpu().tolist() == [301, 200, 65, 1]   # the slot that broke the promise gets no token
+    assert np.isfinite(_np(out)).all()
+    kvc.kvc_get_status()
+
+
 def test_grid_stride_compaction_on_workloads():
     """The grid-stride compaction kernel (forced here; the one-wave kernel is the default)
     gives the same bit-exact packed caches."""
