@@ -37,7 +37,7 @@ UNIT = "tokens/s"
 # DRAM bytes (read + written) per launch of the decode kernel from one ncu capture of the
 # current kernel (cold-cache replay): llama8b 17.24 MB read + 0 written; zigzag cut to 8
 # layers 215.7 + 4.9 MB, scaled to the 32 layers (4x the cached rows, traffic in proportion).
-DECODE_TRAFFIC = {"llama8b": 17.24e6, "zigzag": 4 * (215.7e6 + 4.9e6)}
+DECODE_TRAFFIC = {"llama8b": 17.16e6, "zigzag": 4 * (215.64e6 + 1.67e6)}
 DECODE_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum of one capture of this kernel"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -237,7 +237,8 @@ def cuda_arm(args, wl, rank, world, local_rank):
         pipe.compact_step()
         e[3].record()
         for t in range(n_dec):
-            # one launch per token step: append the new K/V rows and decode (kvc_append_decode)
+            # one launch per token step: append the new K/V rows and decode (kvc_append_decode for
+            # the first, kvc_append_decode_chain after it)
             pipe.decode_step(t, out=out_all[t])
         e[4].record()
 
@@ -342,7 +343,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "decode_hbm_gbs": dec_gbs,
         "score_select_compact_us_per_layer": ssc_us / wl.n_layers,
         "phases": phases,
-        "roofline": {"kernel": "decode_mma_kernel (kvc_append_decode)", "bound": "hbm", "achieved": dec_gbs, "peak": hbm,
+        "roofline": {"kernel": "decode_mma_kernel (kvc_append_decode_chain)", "bound": "hbm", "achieved": dec_gbs, "peak": hbm,
                      "unit": "GB/s", "frac": dec_gbs / hbm, "traffic": DECODE_TRAFFIC.get(wl.name),
                      "traffic_source": DECODE_TRAFFIC_SOURCE if wl.name in DECODE_TRAFFIC else None,
                      "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": dec_bytes},
