@@ -680,7 +680,9 @@ kvc_status launch_select(kvc::SelectParams p, int S, int N, cudaStream_t stream,
       return fail(KVC_ERR_CUDA, "%s: launch: %s", what, cudaGetErrorString(e));
     }
   } else {
-    p.key_cap = kvc::select_key_cap(p.L, p.C);
+    // More slots than SMs: without the key cache two 1024-thread CTAs fit on an SM, so the
+    // slots run in one wave (the scores are re-read from L2 each pass); otherwise cache them.
+    p.key_cap = S > di->sms ? 0 : kvc::select_key_cap(p.L, p.C);
     smem = kvc::select_smem_bytes(p.key_cap);
     if ((rc = set_smem(kvc::select_kernel, smem, what)) != KVC_OK) return rc;
     kvc::select_kernel<<<S, kvc::SEL_THREADS, smem, stream>>>(p);

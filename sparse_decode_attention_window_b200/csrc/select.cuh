@@ -45,6 +45,56 @@ KVC_DEV uint32_t order_key(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// floor(max(v, 0) * 2^fx) as an integer, exactly: the fp32 significand shifted by the
+// scaled exponent (no floating-point rounding). The scale is chosen from the slot's
+// largest score, so every finite weight stays below 2^62 (shift <= 39); larger
+// shifts (an infinite score) saturate.
+KVC_DEV unsigned long long fixed_weight(float v, int fx) {
+  if (!(v > 0.f)) return 0ull;
+  const uint32_t b = __float_as_uint(v);
+  const int e = (int)(b >> 23);                                     // sign bit is 0
+  const unsigned long long m = e ? (unsigned long long)((b & 0x7fffffu) | 0x800000u) : (b & 0x7fffffu);
+  const int sh = (e ? e - 150 : -149) + fx;                          // v = m * 2^(sh - fx)
+  if (sh >= 0) return sh <= 40 ? m << sh : ~0ull;
+  return sh > -64 ? m >> -sh : 0ull;
+}
+
+// Weighted histogram step for the lanes `mm` of a warp that match the current prefix: each
+// group of lanes sharing a bin adds its count and its 64-bit weight sum once. A warp whose
+// matching lanes fall in one or two bins sums each group with warp reductions over three
+// 21-bit limbs (they cannot overflow 32 bits); otherwise (groups are then small) each
+// group's leader adds its lanes' staged weights.
+KVC_DEV void hist_add_weighted(unsigned mm, unsigned peers, uint32_t bin, unsigned long long wt,
+                               uint32_t* hcnt, unsigned long long* hw, unsigned long long* wstage) {
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(peers) - 1;
+  const unsigned leaders = __ballot_sync(mm, lane == leader);
+  unsigned long long sum;
+  if (__popc(leaders) <= 2) {
+    const unsigned a = __reduce_add_sync(peers, (unsigned)(wt & 0x1fffffu));
+    const unsigned b = __reduce_add_sync(peers, (unsigned)((wt >> 21) & 0x1fffffu));
+    const unsigned c = __reduce_add_sync(peers, (unsigned)(wt >> 42));
+    sum = (unsigned long long)a + ((unsigned long long)b << 21) + ((unsigned long long)c << 42);
+  } else {
+    wstage[threadIdx.x] = wt;
+    __syncwarp(mm);
+    sum = 0;
+    if (lane == leader) {
+      unsigned rest = peers;
+      while (rest) {
+        const int l = __ffs(rest) - 1;
+        rest &= rest - 1;
+        sum += wstage[(threadIdx.x & ~31) + l];
+      }
+    }
+    __syncwarp(mm);
+  }
+  if (lane == leader) {
+    atomicAdd(&hcnt[bin], (uint32_t)__popc(peers));
+    atomicAdd(&hw[bin], sum);
+  }
+}
+
 struct SelShared {
   uint32_t hcnt[SEL_MAX_BINS];
   unsigned long long hw[SEL_MAX_BINS];
@@ -166,8 +216,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
   auto weight_of = [&](int n) -> unsigned long long {
     if (chunk) return (unsigned long long)(ce[n] - (n > 0 ? ce[n - 1] : -1));
     if (massc) {
-      float v = fmaxf(sc[n], 0.f);
-      return (unsigned long long)__double2ull_rz(ldexp((double)v, fx));
+      return fixed_weight(sc[n], fx);
     }
     return 1ull;
   };
@@ -205,11 +254,10 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
   // radix passes: digits [31:21], [20:10], [9:0]
   uint32_t prefix = 0, pmask = 0, cnt_above = 0;
   unsigned long long w_above = 0;
-  const int shifts[3] = {21, 10, 0};
-  const int bitsz[3] = {11, 11, 10};
   const int lane = tid & 31;
   for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass], nb = 1 << bitsz[pass];
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nb = pass == 2 ? 1024 : 2048;
     for (int b = tid; b < nb; b += blockDim.x) { sh.hcnt[b] = 0; sh.hw[b] = 0; }
     __syncthreads();
     for (int base = 0; base < N; base += blockDim.x) {
@@ -231,20 +279,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
           // top-B: every weight is 1, the count is the weight
           if (lane == leader) atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
         } else {
-          sh.wstage[tid] = wt;
-          __syncwarp(mm);
-          if (lane == leader) {
-            unsigned long long sum = 0;
-            unsigned rest = peers;
-            while (rest) {
-              int l = __ffs(rest) - 1;
-              rest &= rest - 1;
-              sum += sh.wstage[(tid & ~31) + l];
-            }
-            atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
-            atomicAdd(&sh.hw[bin], sum);
-          }
-          __syncwarp(mm);
+          hist_add_weighted(mm, peers, bin, wt, sh.hcnt, sh.hw, sh.wstage);
         }
       }
     }
@@ -560,8 +595,7 @@ __global__ void __launch_bounds__(SCL_THREADS) select_cluster_kernel(SelectParam
   auto weight_of = [&](int i) -> unsigned long long {
     if (chunk) return wts[i];
     if (massc) {
-      const float v = fmaxf(key_score(keys[i]), 0.f);
-      return (unsigned long long)__double2ull_rz(ldexp((double)v, fx));
+      return fixed_weight(key_score(keys[i]), fx);
     }
     return 1ull;
   };
@@ -598,20 +632,7 @@ __global__ void __launch_bounds__(SCL_THREADS) select_cluster_kernel(SelectParam
         if (unit) {
           if (lane == leader) atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
         } else {
-          sh.wstage[tid] = wt;
-          __syncwarp(mm);
-          if (lane == leader) {
-            unsigned long long sum = 0;
-            unsigned rest = peers;
-            while (rest) {
-              const int l = __ffs(rest) - 1;
-              rest &= rest - 1;
-              sum += sh.wstage[(tid & ~31) + l];
-            }
-            atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
-            atomicAdd(&sh.hw[bin], sum);
-          }
-          __syncwarp(mm);
+          hist_add_weighted(mm, peers, bin, wt, sh.hcnt, sh.hw, sh.wstage);
         }
       }
     }
