@@ -98,3 +98,19 @@ def test_workspace_sizes_are_positive_for_score_and_decode():
     assert kvc.kvc_workspace_size(kvc.KVC_WS_SCORE, sh) > 0
     assert kvc.kvc_workspace_size(kvc.KVC_WS_DECODE, sh) > 0
     assert kvc.kvc_workspace_size(kvc.KVC_WS_SELECT, sh) == 0
+
+
+def test_fused_decode_entries_validate():
+    lib = kvc.library()
+    p = ctypes.c_void_p(16)
+    sh = ctypes.byref(_shape())
+    # the chained form needs its promise array
+    assert lib.kvc_append_decode_chain(sh, p, p, p, p, p, p, p, None, p, 64, p, p, 1 << 20, None) == \
+        _abi.KVC_ERR_INVALID_ARG
+    assert b"stable" in lib.kvc_last_error()
+    assert lib.kvc_append_decode_chain(sh, None, p, p, p, p, p, p, p, p, 64, p, p, 1 << 20, None) == \
+        _abi.KVC_ERR_INVALID_ARG
+    assert lib.kvc_append_decode(sh, p, p, p, p, p, p, None, p, 64, p, p, 1 << 20, None) == _abi.KVC_ERR_INVALID_ARG
+    bad = ctypes.byref(_shape(d=96))
+    assert lib.kvc_append_decode_chain(bad, p, p, p, p, p, p, p, p, p, 64, p, p, 1 << 20, None) == \
+        _abi.KVC_ERR_UNSUPPORTED

@@ -494,15 +494,17 @@ def test_fused_append_decode_overflow_keeps_old_rows():
     kvc.kvc_get_status()
 
 
-@pytest.mark.parametrize("S,counts", [(32, None), (5, [1000, 3, 0, 64, 700]), (70, None)])
-def test_chained_append_decode_is_bit_identical(S, counts):
+@pytest.mark.parametrize("S,counts,G,d", [(32, None, 4, 128), (5, [1000, 3, 0, 64, 700], 4, 128),
+                                          (70, None, 4, 128), (16, None, 8, 128), (12, None, 2, 64)])
+def test_chained_append_decode_is_bit_identical(S, counts, G, d):
     """kvc_append_decode_chain (the kept rows may load before the previous launch ends)
     returns bit for bit what kvc_append_decode returns, step after step, on uniform,
-    ragged and many-slot caches; the results match the oracle."""
+    ragged and many-slot caches, for G = 2, 4, 8 and d = 64, 128; the results match the
+    oracle."""
     import sparse_decode_attention_window_b200 as kvc
-    G, d, steps = 4, 128, 12
+    steps = 12
     g = torch.Generator().manual_seed(S)
-    cnt = (torch.full((S,), 1024, dtype=torch.int32) if counts is None and S <= 32 else
+    cnt = (torch.full((S,), 1024, dtype=torch.int32) if counts is None and S == 32 else
            torch.randint(0, 900, (S,), generator=g, dtype=torch.int32) if counts is None else
            torch.tensor(counts, dtype=torch.int32))
     sh = kvc.make_shape(S, G, d, int(cnt.max()) + steps, 0, S, 1, torch.bfloat16)
