@@ -47,7 +47,7 @@ struct DmCfg {
 // rescale; probabilities then stay below 2^8, far inside fp32 and the bf16 hi/lo split.
 constexpr float DM_LAZY_LOG2 = 8.f;
 constexpr int DM_MIN_TOKENS_PER_CTA = 64;            // token split: no CTA gets less than a tile
-constexpr long long DM_SEG_COST = 128;               // token split: fixed work of one slot segment, in tokens
+constexpr long long DM_SEG_COST = 256;               // token split: fixed work of one slot segment, in tokens
 constexpr int DM_MAX_CLUSTER = 8;
 constexpr int DM_APPENDS = 1 << 30;                  // flag in the per-slot row count: the last row is appended
 
