@@ -364,7 +364,10 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "roofline": {"kernel": "decode_mma_kernel (kvc_append_decode_chain)", "bound": "hbm", "achieved": dec_gbs, "peak": hbm,
                      "unit": "GB/s", "frac": dec_gbs / hbm, "traffic": DECODE_TRAFFIC.get(wl.name),
                      "traffic_source": DECODE_TRAFFIC_SOURCE if wl.name in DECODE_TRAFFIC else None,
-                     "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": dec_bytes},
+                     "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": dec_bytes,
+                     "note": ("the packed cache fits in L2 and is re-read by each decode step, so this "
+                              "fraction measures the launch's latency, not HBM bandwidth"
+                              if dec_bytes < l2 else "cache larger than L2: read from HBM each step")},
         "clocks": clk,
         "gpu_launches": int(launches),
         "launches_per_step": int(launches_per_step),
