@@ -254,7 +254,6 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
   // radix passes: digits [31:21], [20:10], [9:0]
   uint32_t prefix = 0, pmask = 0, cnt_above = 0;
   unsigned long long w_above = 0;
-  const int lane = tid & 31;
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const int nb = pass == 2 ? 1024 : 2048;
@@ -271,16 +270,13 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
         bin = (key >> shift) & (nb - 1);
         if (match) wt = weight_of(n);
       }
-      const unsigned mm = __ballot_sync(0xffffffffu, match);
-      if (match) {
-        const unsigned peers = __match_any_sync(mm, bin);
-        const int leader = __ffs(peers) - 1;
-        if (unit) {
-          // top-B: every weight is 1, the count is the weight
-          if (lane == leader) atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
-        } else {
-          hist_add_weighted(mm, peers, bin, wt, sh.hcnt, sh.hw, sh.wstage);
-        }
+      if (unit) {
+        // top-B: every weight is 1, the count is the weight; one shared atomic per key
+        // (grouping a warp's keys by bin with match.any costs more when they spread)
+        if (match) atomicAdd(&sh.hcnt[bin], 1u);
+      } else {
+        const unsigned mm = __ballot_sync(0xffffffffu, match);
+        if (match) hist_add_weighted(mm, __match_any_sync(mm, bin), bin, wt, sh.hcnt, sh.hw, sh.wstage);
       }
     }
     __syncthreads();
@@ -625,15 +621,11 @@ __global__ void __launch_bounds__(SCL_THREADS) select_cluster_kernel(SelectParam
         bin = (key >> shift) & (nb - 1);
         if (match) wt = weight_of(i);
       }
-      const unsigned mm = __ballot_sync(FULL, match);
-      if (match) {
-        const unsigned peers = __match_any_sync(mm, bin);
-        const int leader = __ffs(peers) - 1;
-        if (unit) {
-          if (lane == leader) atomicAdd(&sh.hcnt[bin], (uint32_t)__popc(peers));
-        } else {
-          hist_add_weighted(mm, peers, bin, wt, sh.hcnt, sh.hw, sh.wstage);
-        }
+      if (unit) {
+        if (match) atomicAdd(&sh.hcnt[bin], 1u);   // top-B: one shared atomic per key
+      } else {
+        const unsigned mm = __ballot_sync(FULL, match);
+        if (match) hist_add_weighted(mm, __match_any_sync(mm, bin), bin, wt, sh.hcnt, sh.hw, sh.wstage);
       }
     }
     cluster_sync();
