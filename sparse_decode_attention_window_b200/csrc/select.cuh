@@ -59,46 +59,21 @@ KVC_DEV unsigned long long fixed_weight(float v, int fx) {
   return sh > -64 ? m >> -sh : 0ull;
 }
 
-// Weighted histogram step for the lanes `mm` of a warp that match the current prefix: each
-// group of lanes sharing a bin adds its count and its 64-bit weight sum once. A warp whose
-// matching lanes fall in one or two bins sums each group with warp reductions over three
-// 21-bit limbs (they cannot overflow 32 bits); otherwise (groups are then small) each
-// group's leader adds its lanes' staged weights.
-KVC_DEV void hist_add_weighted(unsigned mm, unsigned peers, uint32_t bin, unsigned long long wt,
-                               uint32_t* hcnt, unsigned long long* hw, unsigned long long* wstage) {
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(peers) - 1;
-  const unsigned leaders = __ballot_sync(mm, lane == leader);
-  unsigned long long sum;
-  if (__popc(leaders) <= 2) {
-    const unsigned a = __reduce_add_sync(peers, (unsigned)(wt & 0x1fffffu));
-    const unsigned b = __reduce_add_sync(peers, (unsigned)((wt >> 21) & 0x1fffffu));
-    const unsigned c = __reduce_add_sync(peers, (unsigned)(wt >> 42));
-    sum = (unsigned long long)a + ((unsigned long long)b << 21) + ((unsigned long long)c << 42);
-  } else {
-    wstage[threadIdx.x] = wt;
-    __syncwarp(mm);
-    sum = 0;
-    if (lane == leader) {
-      unsigned rest = peers;
-      while (rest) {
-        const int l = __ffs(rest) - 1;
-        rest &= rest - 1;
-        sum += wstage[(threadIdx.x & ~31) + l];
-      }
-    }
-    __syncwarp(mm);
-  }
-  if (lane == leader) {
-    atomicAdd(&hcnt[bin], (uint32_t)__popc(peers));
-    atomicAdd(&hw[bin], sum);
-  }
+// Adds a 64-bit weight to a bin kept as two 32-bit words, with one shared atomic per
+// word: the low word's atomic returns its old value, so the addition that wraps it is
+// known and carries one into the high word. Exact for any number of keys (the low word
+// wraps as often as the true sum crosses a multiple of 2^32, and each wrap is counted
+// once). Per key, so no grouping of a warp's keys by bin is needed.
+KVC_DEV void bin_add_u64(uint32_t* lo, uint32_t* hi, unsigned long long w) {
+  const uint32_t wl = (uint32_t)w, wh = (uint32_t)(w >> 32);
+  const uint32_t old = atomicAdd(lo, wl);
+  const uint32_t up = wh + (old + wl < old ? 1u : 0u);
+  if (up) atomicAdd(hi, up);
 }
 
 struct SelShared {
   uint32_t hcnt[SEL_MAX_BINS];
-  unsigned long long hw[SEL_MAX_BINS];
-  unsigned long long wstage[SEL_THREADS];
+  uint32_t hwl[SEL_MAX_BINS], hwh[SEL_MAX_BINS];   // bin weights, low and high 32 bits
   unsigned long long scan64[33];
   uint32_t scan32[33];
   // results of the bin search
@@ -257,7 +232,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const int nb = pass == 2 ? 1024 : 2048;
-    for (int b = tid; b < nb; b += blockDim.x) { sh.hcnt[b] = 0; sh.hw[b] = 0; }
+    for (int b = tid; b < nb; b += blockDim.x) { sh.hcnt[b] = 0; sh.hwl[b] = 0; sh.hwh[b] = 0; }
     __syncthreads();
     for (int base = 0; base < N; base += blockDim.x) {
       const int n = base + tid;
@@ -270,13 +245,12 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
         bin = (key >> shift) & (nb - 1);
         if (match) wt = weight_of(n);
       }
-      if (unit) {
-        // top-B: every weight is 1, the count is the weight; one shared atomic per key
-        // (grouping a warp's keys by bin with match.any costs more when they spread)
-        if (match) atomicAdd(&sh.hcnt[bin], 1u);
-      } else {
-        const unsigned mm = __ballot_sync(0xffffffffu, match);
-        if (match) hist_add_weighted(mm, __match_any_sync(mm, bin), bin, wt, sh.hcnt, sh.hw, sh.wstage);
+      // one shared atomic per key and word (grouping a warp's keys by bin with match.any
+      // costs more when they spread over many bins); top-B: every weight is 1, the count
+      // is the weight
+      if (match) {
+        atomicAdd(&sh.hcnt[bin], 1u);
+        if (!unit) bin_add_u64(&sh.hwl[bin], &sh.hwh[bin], wt);
       }
     }
     __syncthreads();
@@ -286,7 +260,10 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     const int lo = max(hi - per, 0);
     unsigned long long my_w = 0;
     uint32_t my_c = 0;
-    for (int b = hi - 1; b >= lo; --b) { my_w += unit ? sh.hcnt[b] : sh.hw[b]; my_c += sh.hcnt[b]; }
+    auto bin_w = [&](int b) -> unsigned long long {
+      return unit ? (unsigned long long)sh.hcnt[b] : ((unsigned long long)sh.hwh[b] << 32) | sh.hwl[b];
+    };
+    for (int b = hi - 1; b >= lo; --b) { my_w += bin_w(b); my_c += sh.hcnt[b]; }
     unsigned long long tot_w;
     uint32_t tot_c;
     unsigned long long before_w = block_exclusive_scan<unsigned long long>(hi > lo ? my_w : 0ull, sh.scan64, &tot_w);
@@ -296,7 +273,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
       uint32_t runc = before_c;
       for (int b = hi - 1; b >= lo; --b) {
         const uint32_t cb = sh.hcnt[b];
-        const unsigned long long wb = unit ? (unsigned long long)cb : sh.hw[b];
+        const unsigned long long wb = bin_w(b);
         if (cb > 0 && run < target && run + wb >= target) {
           sh.sel_bin = b;
           sh.w_above_bin = run;
@@ -319,7 +296,8 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
   if (massc) {
     if (tid == 0) {
       // every tied key has the same weight
-      unsigned long long wt = sh.hw[sh.sel_bin] / sh.hcnt[sh.sel_bin];
+      const unsigned long long bw = ((unsigned long long)sh.hwh[sh.sel_bin] << 32) | sh.hwl[sh.sel_bin];
+      unsigned long long wt = bw / sh.hcnt[sh.sel_bin];
       unsigned long long take = (need + wt - 1) / wt;
       a.count[s] = (int)(cnt_above + take);
     }
@@ -414,11 +392,10 @@ constexpr int SCL_IT = 4;       // consecutive keys per thread in an emission ti
 
 struct SelClShared {
   uint32_t hcnt[SEL_MAX_BINS];                 // histogram of this CTA's key range
-  unsigned long long hw[SEL_MAX_BINS];
+  uint32_t hwl[SEL_MAX_BINS], hwh[SEL_MAX_BINS];   // bin weights, low and high 32 bits
   // the owned bin slice summed over the cluster, in descending bin order (t = 0: highest)
   uint32_t mc[SEL_MAX_BINS / 2], pc[SEL_MAX_BINS / 2];
   unsigned long long mw[SEL_MAX_BINS / 2], pw[SEL_MAX_BINS / 2];
-  unsigned long long wstage[SCL_THREADS];
   unsigned long long scan64[33];
   uint32_t scan32[33];
   // values the other ranks read
@@ -606,7 +583,8 @@ __global__ void __launch_bounds__(SCL_THREADS) select_cluster_kernel(SelectParam
     const int sl = nb / K;                      // bins per slice (>= 64)
     for (int b = tid; b < nb; b += nthr) {
       sh.hcnt[b] = 0;
-      sh.hw[b] = 0;
+      sh.hwl[b] = 0;
+      sh.hwh[b] = 0;
     }
     __syncthreads();
     // 1. histogram of this range
@@ -621,11 +599,9 @@ __global__ void __launch_bounds__(SCL_THREADS) select_cluster_kernel(SelectParam
         bin = (key >> shift) & (nb - 1);
         if (match) wt = weight_of(i);
       }
-      if (unit) {
-        if (match) atomicAdd(&sh.hcnt[bin], 1u);   // top-B: one shared atomic per key
-      } else {
-        const unsigned mm = __ballot_sync(FULL, match);
-        if (match) hist_add_weighted(mm, __match_any_sync(mm, bin), bin, wt, sh.hcnt, sh.hw, sh.wstage);
+      if (match) {                     // one shared atomic per key and word (as select_kernel)
+        atomicAdd(&sh.hcnt[bin], 1u);
+        if (!unit) bin_add_u64(&sh.hwl[bin], &sh.hwh[bin], wt);
       }
     }
     cluster_sync();
@@ -644,7 +620,9 @@ __global__ void __launch_bounds__(SCL_THREADS) select_cluster_kernel(SelectParam
         const int b = (r + 1) * sl - 1 - t;
         for (int q = 0; q < K; ++q) {
           c[j] += ld_cluster_u32(map_to_rank(&sh.hcnt[b], q));
-          if (!unit) w[j] += ld_cluster_u64(map_to_rank(&sh.hw[b], q));
+          if (!unit)
+            w[j] += ((unsigned long long)ld_cluster_u32(map_to_rank(&sh.hwh[b], q)) << 32) |
+                    ld_cluster_u32(map_to_rank(&sh.hwl[b], q));
         }
         if (unit) w[j] = c[j];
         my_c += c[j];
