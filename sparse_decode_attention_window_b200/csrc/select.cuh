@@ -196,21 +196,9 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     return 1ull;
   };
 
-  // target
-  unsigned long long target;
-  if (massc) {
-    unsigned long long tw = 0;
-    for (int n = tid; n < N; n += blockDim.x) tw += weight_of(n);
-    unsigned long long total = block_sum<unsigned long long>(tw, sh.scan64);
-    if (total == 0) {           // no mass at all: the first key alone reaches 0.9 * 0
-      if (tid == 0) a.count[s] = 1;
-      return;
-    }
-    double t = ceil((double)a.mass * (double)total);
-    target = (unsigned long long)t;
-    if (target == 0) target = 1;
-    if (target > total) target = total;
-  } else {
+  // target (MASS_COUNT: from the total weight, which the first radix pass sums)
+  unsigned long long target = 0;
+  if (!massc) {
     long long want = a.budget[s];
     long long full = chunk ? (long long)L : (long long)N;
     if (want >= full || want <= 0) {
@@ -268,6 +256,16 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     uint32_t tot_c;
     unsigned long long before_w = block_exclusive_scan<unsigned long long>(hi > lo ? my_w : 0ull, sh.scan64, &tot_w);
     uint32_t before_c = block_exclusive_scan<uint32_t>(hi > lo ? my_c : 0u, sh.scan32, &tot_c);
+    if (massc && pass == 0) {
+      // every key is in the first pass's histogram: tot_w is the slot's total weight
+      if (tot_w == 0) {           // no mass at all: the first key alone reaches 0.9 * 0
+        if (tid == 0) a.count[s] = 1;
+        return;
+      }
+      target = (unsigned long long)ceil((double)a.mass * (double)tot_w);
+      if (target == 0) target = 1;
+      if (target > tot_w) target = tot_w;
+    }
     {
       unsigned long long run = w_above + before_w;
       uint32_t runc = before_c;
