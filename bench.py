@@ -292,6 +292,15 @@ def cuda_arm(args, wl, rank, world, local_rank):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_step_max = float(t.item())
 
+    # ---- labelled aside (not the metric): the same steps back to back with no L2 flush, so
+    # the inputs the previous replay left in L2 stay there
+    warm_ms = []
+    for _ in range(min(5, args.steps)):
+        graph.replay()
+        torch.cuda.synchronize()
+        warm_ms.append(e[0].elapsed_time(e[4]))
+    kvc.kvc_get_status()
+
     # ---- end to end through the public API with host buffers: a second pipeline (own
     # inputs, cache and outputs) so consecutive steps can overlap their copies and compute
     inp2 = make_inputs(wl_r, dev)
@@ -375,6 +384,9 @@ def cuda_arm(args, wl, rank, world, local_rank):
                   "external CUDA events captured between the phases; decode per launch = the 64-launch "
                   "loop time / launches",
         "e2e": e2e,
+        "warm_l2": {"ms_per_step": statistics.mean(warm_ms), "steps": len(warm_ms),
+                    "note": "no L2 flush between steps (inputs partly L2-resident); not the metric"},
+        "ms_per_step_median": statistics.median(step_ms),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
