@@ -430,6 +430,46 @@ def test_maximum_slot_counts(G, S, fused):
         assert (_np(ln) == _np(count) + 1).all()
 
 
+@pytest.mark.parametrize("name,kw", [("llama8b", {}), ("fastgen", dict(batch=2, L=6000, steps=24)),
+                                     ("zigzag", dict(n_layers=6, L=8192, steps=12))])
+def test_graph_replay_of_a_step_matches_eager(name, kw):
+    """The step as the benchmark runs it - score, select, compact and the decode loop
+    (chained steps, programmatic dependent launch) captured once in a CUDA graph and
+    replayed twice - gives bit for bit the outputs of the same calls made eagerly."""
+    from sparse_decode_attention_window_b200.pipeline import KvcPipeline
+    import sparse_decode_attention_window_b200 as kvc
+    wl = get(name).scaled(**kw) if kw else get(name)
+    inp = make_inputs(wl, "cuda")
+    pipe = KvcPipeline(wl, inp)
+    outs = torch.empty((wl.steps,) + tuple(pipe.out.shape), dtype=torch.float32, device="cuda")
+
+    def step():
+        pipe.compress()
+        for t in range(wl.steps):
+            pipe.decode_step(t, out=outs[t])
+
+    step()
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    eager = outs.clone()
+    idx_eager, cnt_eager = pipe.idx.clone(), pipe.count.clone()
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=cs):
+        step()
+    torch.cuda.current_stream().wait_stream(cs)
+    for _ in range(2):
+        outs.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        kvc.kvc_get_status()
+        assert torch.equal(pipe.count, cnt_eager)
+        assert torch.equal(pipe.idx, idx_eager)
+        assert torch.equal(outs, eager), f"max diff {(outs - eager).abs().max().item():.3e}"
+    del g
+
+
 def test_wide_window_takes_cuda_core_scoring_path():
     """G*w = 256 rows exceeds the tensor-core tile: scoring runs on the CUDA-core kernels;
     decode with G = 8 query heads per KV head."""
