@@ -480,7 +480,9 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
   // Fused append: every CTA has read len once it gets here. Its ticket is taken now (a
   // release: the CTA's reads of len come first; no acquire, so warp 0 does not wait for
   // it) but only looked at when the CTA ends; the CTA that drew the last ticket then
-  // publishes the new lengths (nothing in this launch reads len after this point).
+  // publishes the new lengths (nothing in this launch reads len after this point). The
+  // ticket stays on a consumer thread: drawn in the producer warp, chained steps measured
+  // wrong lengths (cause not found).
   int ticket = -1;
   if (a.append && tid == 0)
     asm volatile("atom.release.gpu.global.add.s32 %0, [%1], 1;" : "=r"(ticket) : "l"(&a.counters[S]), "r"(1) : "memory");
