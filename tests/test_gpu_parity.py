@@ -295,6 +295,34 @@ def test_chunk_selection_over_slot_counts(S, C, n_local):
         np.testing.assert_array_equal(idx[s, :cnt[s]].astype(np.int64), want, err_msg=f"slot {s}")
 
 
+@pytest.mark.parametrize("S", [4, 150])
+def test_selection_flags_bad_policies_and_keeps_the_other_slots(S):
+    """An unknown policy code, and SPECIAL without a special mask, keep nothing for that slot
+    and set the index-range flag; the other slots of the launch (clusters of CTAs for few
+    slots, one CTA per slot for many) are still exact."""
+    import sparse_decode_attention_window_b200 as kvc
+    N = 2048
+    g = torch.Generator().manual_seed(S)
+    sc = torch.rand((S, N), generator=g).float()
+    pol = torch.full((S,), kvc.KVC_POL_TOPB, dtype=torch.int8)
+    pol[1] = 9                                     # not a policy
+    pol[2] = kvc.KVC_POL_SPECIAL                   # needs a special mask: none given
+    bud = torch.full((S,), 100, dtype=torch.int32)
+    sh = kvc.make_shape(S, 1, 64, N, 1, 1, S, torch.bfloat16)
+    idx = torch.full((S, N), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((S,), -1, dtype=torch.int32, device="cuda")
+    kvc.kvc_select(sh, sc.cuda(), pol.cuda(), bud.cuda(), idx, cnt, mass=0.9)
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.kvc_get_status()
+    assert "index-out-of-range" in str(e.value) and "wait-timeout" not in str(e.value)
+    c, ix = _np(cnt), _np(idx)
+    assert c[1] == 0 and c[2] == 0
+    for s in [0] + list(range(3, S)):
+        np.testing.assert_array_equal(ix[s, :c[s]].astype(np.int64), O.top_b(sc[s].double().numpy(), 100),
+                                      err_msg=f"slot {s}")
+    kvc.kvc_get_status()
+
+
 def test_one_cta_per_slot_selection_on_workloads():
     """Selection at one CTA per slot (forced here; few slots take thread-block clusters by
     default) passes the same oracle checks."""
