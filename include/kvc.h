@@ -332,6 +332,16 @@ const char* kvc_version(void);
 /* Number of kernels this library has launched in this process so far (diagnostic). */
 unsigned long long kvc_launch_count(void);
 
+/*
+ * kvc_check_wait_limit - diagnostic of the library's failure path: launches one CTA whose
+ *   thread waits on an mbarrier that nothing arrives on, with the bounded wait every
+ *   pipeline in the library uses (they give up after 2 s; here after limit_us). The wait
+ *   gives up, sets KVC_DEVERR_WAIT_TIMEOUT and the kernel returns, so kvc_get_status then
+ *   reports the timeout and the context stays usable. limit_us in [1, 1e6], else
+ *   KVC_ERR_INVALID_ARG.
+ */
+kvc_status kvc_check_wait_limit(int32_t limit_us, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -19,7 +19,7 @@ from ._abi import (KvcShape, KvcError, KVC_BF16, KVC_FP32, KVC_POL_TOPB, KVC_POL
 __all__ = ["KvcShape", "KvcError", "make_shape", "kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout",
            "kvc_compact", "kvc_append", "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_version",
            "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_append_decode_chain", "kvc_select_chunks",
-           "kvc_retained_mass", "kvc_profile_heads", "kvc_append_window",
+           "kvc_retained_mass", "kvc_profile_heads", "kvc_append_window", "kvc_check_wait_limit",
            "library", "KVC_BF16", "KVC_FP32", "KVC_POL_TOPB", "KVC_POL_MASS_COUNT", "KVC_POL_LOCAL",
            "KVC_POL_SPECIAL", "KVC_POL_FULL", "KVC_POL_CHUNK", "KVC_WS_SCORE", "KVC_WS_SELECT", "KVC_WS_DECODE"]
 
@@ -149,6 +149,12 @@ def kvc_profile_heads(shape, score, policy, window, tau=0.95, special_mask=None,
     _check("kvc_profile_heads",
            library().kvc_profile_heads(ctypes.byref(shape), _ptr(score), _ptr(special_mask), int(window),
                                        float(tau), _ptr(policy), _ptr(shares), _stream(stream)))
+
+
+def kvc_check_wait_limit(limit_us, stream=None):
+    """Diagnostic: a kernel waits on a barrier nothing arrives on until limit_us, gives up and
+    flags a wait timeout (see include/kvc.h)."""
+    _check("kvc_check_wait_limit", library().kvc_check_wait_limit(int(limit_us), _stream(stream)))
 
 
 def kvc_get_status(stream=None):

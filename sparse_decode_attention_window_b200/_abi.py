@@ -23,7 +23,7 @@ EXPORTS = ["kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout", "kvc_co
            "kvc_append_window",
            "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_last_error", "kvc_version",
            "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_append_decode_chain", "kvc_select_chunks",
-           "kvc_retained_mass", "kvc_profile_heads"]
+           "kvc_retained_mass", "kvc_profile_heads", "kvc_check_wait_limit"]
 
 
 class KvcShape(ctypes.Structure):
@@ -73,6 +73,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "kvc_select_chunks": (i32, [sh, vp, vp, i32, vp, i32, vp, i32, vp, vp]),
         "kvc_retained_mass": (i32, [sh, vp, i32, vp, i32, vp, vp, vp]),
         "kvc_profile_heads": (i32, [sh, vp, vp, i32, f32, vp, vp, vp]),
+        "kvc_check_wait_limit": (i32, [i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

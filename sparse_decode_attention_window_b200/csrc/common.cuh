@@ -131,19 +131,20 @@ KVC_DEV uint64_t global_timer_ns() {
 #define KVC_WAIT_LIMIT_NS 2000000000ull
 #endif
 
-KVC_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
+KVC_DEV bool mbar_wait_limit(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > KVC_WAIT_LIMIT_NS) {
+    if (global_timer_ns() - t0 > limit_ns) {
       kvc_flag(KVC_DEVERR_WAIT_TIMEOUT);
       return false;
     }
   }
 }
+KVC_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) { return mbar_wait_limit(bar, parity, KVC_WAIT_LIMIT_NS); }
 
 // ---------------------------------------------------------------- thread-block clusters
 KVC_DEV uint32_t cluster_rank() {

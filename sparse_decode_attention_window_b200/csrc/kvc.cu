@@ -723,6 +723,29 @@ kvc_status kvc_select(const kvc_shape* shape, const float* score, const int8_t* 
   return launch_select(p, shape->n_slots, std::max(shape->L, p.C), stream, "kvc_select");
 }
 
+namespace kvc {
+// One thread waits on a barrier that nothing arrives on, with the same bounded wait every
+// pipeline of the library uses (only the limit differs): it gives up, flags the timeout and
+// the kernel returns.
+__global__ void wait_limit_probe_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, limit_ns);
+}
+}  // namespace kvc
+
+kvc_status kvc_check_wait_limit(int32_t limit_us, cudaStream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000)
+    return fail(KVC_ERR_INVALID_ARG, "kvc_check_wait_limit: limit_us = %d not in [1, 1e6]", limit_us);
+  kvc::wait_limit_probe_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_us * 1000ull);
+  count_launches(1);
+  return check_launch("kvc_check_wait_limit");
+}
+
 kvc_status kvc_alloc_budgets(const int32_t* counts, int32_t n_layers, int32_t spl, int32_t L, int32_t avg_B,
                              int32_t floor_B, int32_t* budgets, int32_t* slot_budgets, cudaStream_t stream) {
   if (!counts || !budgets) return fail(KVC_ERR_INVALID_ARG, "kvc_alloc_budgets: counts and budgets must be non-NULL");

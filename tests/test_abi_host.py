@@ -100,6 +100,13 @@ def test_workspace_sizes_are_positive_for_score_and_decode():
     assert kvc.kvc_workspace_size(kvc.KVC_WS_SELECT, sh) == 0
 
 
+def test_wait_limit_check_validates_its_limit():
+    lib = kvc.library()
+    for bad in (0, -5, 1000001):
+        assert lib.kvc_check_wait_limit(bad, None) == _abi.KVC_ERR_INVALID_ARG
+        assert b"limit_us" in lib.kvc_last_error()
+
+
 def test_fused_decode_entries_validate():
     lib = kvc.library()
     p = ctypes.c_void_p(16)

@@ -323,6 +323,32 @@ def test_selection_flags_bad_policies_and_keeps_the_other_slots(S):
     kvc.kvc_get_status()
 
 
+def test_bounded_wait_gives_up_and_leaves_the_context_usable():
+    """A wait on a barrier that nothing arrives on ends after its limit with the wait-timeout
+    flag; the next status read is clean and the next library call is exact."""
+    import sparse_decode_attention_window_b200 as kvc
+    limit_us = 2000
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    kvc.kvc_check_wait_limit(limit_us)
+    t1.record()
+    with pytest.raises(kvc.KvcError) as e:
+        kvc.kvc_get_status()
+    assert "wait-timeout" in str(e.value) and "index-out-of-range" not in str(e.value)
+    assert limit_us * 1e-3 <= t0.elapsed_time(t1) < 1000.0
+    kvc.kvc_get_status()
+    S, N = 4, 4096
+    sc = torch.rand((S, N), generator=torch.Generator().manual_seed(5)).float()
+    sh = kvc.make_shape(S, 1, 64, N, 1, 1, S, torch.bfloat16)
+    idx = torch.full((S, N), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(S, dtype=torch.int32, device="cuda")
+    kvc.kvc_select(sh, sc.cuda(), torch.full((S,), kvc.KVC_POL_TOPB, dtype=torch.int8, device="cuda"),
+                   torch.full((S,), 300, dtype=torch.int32, device="cuda"), idx, cnt)
+    kvc.kvc_get_status()
+    for s in range(S):
+        np.testing.assert_array_equal(_np(idx)[s, :300].astype(np.int64), O.top_b(sc[s].double().numpy(), 300))
+
+
 def test_one_cta_per_slot_selection_on_workloads():
     """Selection at one CTA per slot (forced here; few slots take thread-block clusters by
     default) passes the same oracle checks."""
