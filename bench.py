@@ -230,24 +230,30 @@ def cuda_arm(args, wl, rank, world, local_rank):
     n_dec = wl.steps
     out_all = torch.empty((n_dec,) + tuple(pipe.out.shape), dtype=torch.float32, device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
-    e = [ev() for _ in range(5)]
+    e = [ev() for _ in range(5)]      # phase boundaries (the phase graph)
+    ew = [ev(), ev()]                 # the step's two ends (the timed graph)
 
-    def step_calls():
-        # one whole step of the hot path; the timing events become graph nodes. The decode
-        # loop carries events only at its two ends so consecutive launches keep overlapping
-        # (programmatic dependent launch); its per-launch time is the loop time / steps.
-        e[0].record()
+    def step_calls(phases=False):
+        # one whole step of the hot path; the timing events become graph nodes. The timed graph
+        # carries events only at the step's two ends, so every launch may overlap the end of the
+        # one before it (programmatic dependent launch); the phase graph adds events between the
+        # phases (which ends that overlap there) and times each phase. The decode loop carries
+        # none inside: its per-launch time is the loop time / steps.
+        (e[0] if phases else ew[0]).record()
         pipe.score_step()
-        e[1].record()
+        if phases:
+            e[1].record()
         pipe.select_step()
-        e[2].record()
+        if phases:
+            e[2].record()
         pipe.compact_step()
-        e[3].record()
+        if phases:
+            e[3].record()
         for t in range(n_dec):
             # one launch per token step: append the new K/V rows and decode (kvc_append_decode for
             # the first, kvc_append_decode_chain after it)
             pipe.decode_step(t, out=out_all[t])
-        e[4].record()
+        (e[4] if phases else ew[1]).record()
 
     # eager warm-up: loads every kernel and sets its attributes before capture
     for _ in range(max(1, args.warmup)):
@@ -258,18 +264,24 @@ def cuda_arm(args, wl, rank, world, local_rank):
     counts = pipe.count.cpu().numpy()
     work = work_per_step(wl, counts, pipe.C)
 
-    # the whole step as one CUDA graph (launch-bound decode loop: 2 launches per token step)
+    # the whole step as one CUDA graph (launch-bound decode loop: one launch per token step),
+    # and the same step with phase events
     graph = torch.cuda.CUDAGraph()
+    graph_ph = torch.cuda.CUDAGraph()
     cap_stream = torch.cuda.Stream(device=dev)
     cap_stream.wait_stream(torch.cuda.current_stream())
     n0 = kvc.kvc_launch_count()
     with torch.cuda.graph(graph, stream=cap_stream):
         step_calls()
     launches_per_step = kvc.kvc_launch_count() - n0
+    with torch.cuda.graph(graph_ph, stream=cap_stream):
+        step_calls(phases=True)
     torch.cuda.current_stream().wait_stream(cap_stream)
     for _ in range(args.warmup):
         flush_l2()
         graph.replay()
+        flush_l2()
+        graph_ph.replay()
     torch.cuda.synchronize()
     kvc.kvc_get_status()
 
@@ -277,20 +289,29 @@ def cuda_arm(args, wl, rank, world, local_rank):
     clocks.start()
     barrier()
     torch.cuda.synchronize()
-    step_ms, score_ms, select_ms, compact_ms, dec_ms = [], [], [], [], []
+    step_ms = []
     for _ in range(args.steps):
         flush_l2()             # L2 flushed between steps, outside the timed events
         graph.replay()
         torch.cuda.synchronize()
-        score_ms.append(e[0].elapsed_time(e[1]))
-        select_ms.append(e[1].elapsed_time(e[2]))
-        compact_ms.append(e[2].elapsed_time(e[3]))
-        step_ms.append(e[0].elapsed_time(e[4]))
-        dec_ms.append(e[3].elapsed_time(e[4]) / max(n_dec, 1))
+        step_ms.append(ew[0].elapsed_time(ew[1]))
     torch.cuda.synchronize()
     barrier()
     launches = launches_per_step * args.steps
     clk = clocks.stop()
+    kvc.kvc_get_status()
+
+    # ---- the phase breakdown, from the graph with phase events (not the metric)
+    score_ms, select_ms, compact_ms, dec_ms, ph_step_ms = [], [], [], [], []
+    for _ in range(min(args.steps, 10)):
+        flush_l2()
+        graph_ph.replay()
+        torch.cuda.synchronize()
+        score_ms.append(e[0].elapsed_time(e[1]))
+        select_ms.append(e[1].elapsed_time(e[2]))
+        compact_ms.append(e[2].elapsed_time(e[3]))
+        ph_step_ms.append(e[0].elapsed_time(e[4]))
+        dec_ms.append(e[3].elapsed_time(e[4]) / max(n_dec, 1))
     kvc.kvc_get_status()
 
     ms_step = statistics.mean(step_ms)
@@ -305,7 +326,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
     for _ in range(min(5, args.steps)):
         graph.replay()
         torch.cuda.synchronize()
-        warm_ms.append(e[0].elapsed_time(e[4]))
+        warm_ms.append(ew[0].elapsed_time(ew[1]))
     kvc.kvc_get_status()
 
     # ---- end to end through the public API with host buffers: a second pipeline (own
@@ -338,7 +359,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
                "sample": f"{done} of {wl.n_slots} slots (score, select, {wl.steps} decode steps each) in "
                          f"{dt:.1f} s on 1 thread, scaled to the whole step ({full:.1f} s)"}
 
-    del graph
+    del graph, graph_ph
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -357,6 +378,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "select_us": 1000.0 * statistics.mean(select_ms),
         "compact_us": 1000.0 * statistics.mean(compact_ms),
         "append_decode_us_mean": dec_us,
+        "step_ms_with_phase_events": statistics.mean(ph_step_ms),
     }
     if "score_bytes" in work:
         s_us = phases["score_us"]
@@ -388,9 +410,10 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "clocks": clk,
         "gpu_launches": int(launches),
         "launches_per_step": int(launches_per_step),
-        "timing": "each step is one CUDA-graph replay of the C-ABI calls; phase and per-launch times from "
-                  "external CUDA events captured between the phases; decode per launch = the 64-launch "
-                  "loop time / launches",
+        "timing": "each step is one CUDA-graph replay of the C-ABI calls, timed by external CUDA events "
+                  "at its two ends; phase and per-launch times from a second graph of the same calls with "
+                  "events between the phases (which stop launches overlapping there); decode per launch = "
+                  "the 64-launch loop time / launches",
         "e2e": e2e,
         "warm_l2": {"ms_per_step": statistics.mean(warm_ms), "steps": len(warm_ms),
                     "note": "no L2 flush between steps (inputs partly L2-resident); not the metric"},
