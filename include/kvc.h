@@ -9,6 +9,7 @@
  *   kvc_alloc_budgets  ZigZagKV bounded per-layer budgets from the LMBA counts
  *   kvc_layout         packed-cache offsets and capacities
  *   kvc_compact        gather of the kept rows into the packed per-head cache
+ *   kvc_layout_compact the two above in one launch
  *   kvc_append         one new token per slot per decode step
  *   kvc_decode_attn    split-K GQA decode attention over the ragged packed cache
  *   kvc_append_decode  the two above fused into one launch (the per-step call)
@@ -180,6 +181,18 @@ kvc_status kvc_compact(const kvc_shape* shape, const void* k, const void* v,
                        const int32_t* idx, int32_t max_sel, const int32_t* count,
                        const int64_t* off, void* kp, void* vp, int64_t kp_rows,
                        int32_t* len, cudaStream_t stream);
+
+/*
+ * kvc_layout_compact - kvc_layout followed by kvc_compact, in one launch when
+ *   n_slots <= 512 (every CTA of the compaction scans the capacities itself), else
+ *   as those two launches. Same arguments and results as the two calls: off [S+1]
+ *   int64 and cap [S] int32 are outputs here, with reserve >= 0 as in kvc_layout;
+ *   the rows written, len and the flags are those of kvc_compact.
+ */
+kvc_status kvc_layout_compact(const kvc_shape* shape, const void* k, const void* v,
+                              const int32_t* idx, int32_t max_sel, const int32_t* count,
+                              int32_t reserve, int64_t* off, int32_t* cap, void* kp, void* vp,
+                              int64_t kp_rows, int32_t* len, cudaStream_t stream);
 
 /*
  * kvc_append - one new token per slot: kp[off[s] + len[s]] = k_new[s], vp

@@ -17,7 +17,7 @@ from ._abi import (KvcShape, KvcError, KVC_BF16, KVC_FP32, KVC_POL_TOPB, KVC_POL
                    KVC_POL_SPECIAL, KVC_POL_FULL, KVC_POL_CHUNK, KVC_WS_SCORE, KVC_WS_SELECT, KVC_WS_DECODE)
 
 __all__ = ["KvcShape", "KvcError", "make_shape", "kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout",
-           "kvc_compact", "kvc_append", "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_version",
+           "kvc_compact", "kvc_layout_compact", "kvc_append", "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_version",
            "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_append_decode_chain", "kvc_select_chunks",
            "kvc_retained_mass", "kvc_profile_heads", "kvc_append_window", "kvc_check_wait_limit",
            "library", "KVC_BF16", "KVC_FP32", "KVC_POL_TOPB", "KVC_POL_MASS_COUNT", "KVC_POL_LOCAL",
@@ -86,6 +86,14 @@ def kvc_compact(shape, k, v, idx, count, off, kp, vp, length, stream=None):
     _check("kvc_compact", library().kvc_compact(ctypes.byref(shape), _ptr(k), _ptr(v), _ptr(idx), int(idx.shape[-1]),
                                                 _ptr(count), _ptr(off), _ptr(kp), _ptr(vp), int(kp.shape[0]),
                                                 _ptr(length), _stream(stream)))
+
+
+def kvc_layout_compact(shape, k, v, idx, count, reserve, off, cap, kp, vp, length, stream=None):
+    """kvc_layout then kvc_compact, in one launch for up to 512 slots (see include/kvc.h)."""
+    _check("kvc_layout_compact",
+           library().kvc_layout_compact(ctypes.byref(shape), _ptr(k), _ptr(v), _ptr(idx), int(idx.shape[-1]),
+                                        _ptr(count), int(reserve), _ptr(off), _ptr(cap), _ptr(kp), _ptr(vp),
+                                        int(kp.shape[0]), _ptr(length), _stream(stream)))
 
 
 def kvc_append_window(shape, k_new, v_new, off, cap, length, window, head, kp, vp, stream=None):

@@ -122,34 +122,78 @@ KVC_DEV int warp_slot_search(const int64_t* __restrict__ off, int S, long long x
   return lo;
 }
 
-template <int TPR>
+//
+// LAYOUT (S <= CP_MAX_SLOTS): the layout is computed here as well, in one launch: every CTA
+// scans the capacities round_up(count + reserve, 16) into shared memory itself, and CTA 0
+// also writes them out (off_out, cap_out), so the copy no longer waits for a layout kernel.
+template <int TPR, bool LAYOUT>
 __global__ void __launch_bounds__(CP_THREADS, 4) compact_wave_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, const int32_t* __restrict__ idx, int max_sel,
     const int32_t* __restrict__ count, const int64_t* __restrict__ off, int S, int L, uint4* __restrict__ kp,
-    uint4* __restrict__ vp, int64_t kp_rows, int32_t* __restrict__ len) {
+    uint4* __restrict__ vp, int64_t kp_rows, int32_t* __restrict__ len, int reserve, int64_t* __restrict__ off_out,
+    int32_t* __restrict__ cap_out) {
   __shared__ long long s_off[CP_MAX_SLOTS + 1];
   __shared__ int s_cnt[CP_MAX_SLOTS];
   __shared__ long long src_row[CP_THREADS];   // source row s * L + j, or -1: not written
   __shared__ int s_first_sh, s_last_sh;
+  __shared__ unsigned long long scan_sh[32];
   const int tid = threadIdx.x;
   for (long long s = (long long)blockIdx.x * blockDim.x + tid; s < S; s += (long long)gridDim.x * blockDim.x)
     len[s] = min(max(count[s], 0), max_sel);
-  const long long total = off[S];
+  long long total;
+  int s_first, ns;
+  bool staged;
+  if (LAYOUT) {
+    // the same arithmetic as layout_kernel, over all S slots
+    const bool writer = blockIdx.x == 0;
+    unsigned long long carry = 0;
+    for (int base = 0; base < S; base += CP_THREADS) {
+      const int s = base + tid;
+      unsigned long long c = 0;
+      if (s < S) {
+        const int cs = count[s];
+        c = (unsigned long long)(((long long)max(cs, 0) + reserve + 15) / 16 * 16);
+        s_cnt[s] = min(cs, max_sel);
+        if (writer) cap_out[s] = (int32_t)c;
+      }
+      unsigned long long tot;
+      const unsigned long long before = carry + block_exclusive_scan<unsigned long long>(c, scan_sh, &tot);
+      if (s < S) {
+        s_off[s] = (long long)before;
+        if (writer) off_out[s] = (int64_t)before;
+      }
+      carry += tot;
+    }
+    if (tid == 0) {
+      s_off[S] = (long long)carry;
+      if (writer) off_out[S] = (int64_t)carry;
+    }
+    __syncthreads();
+    total = s_off[S];
+    s_first = 0;
+    ns = S;
+    staged = true;
+  } else {
+    total = off[S];
+  }
   const long long r0 = total * blockIdx.x / gridDim.x, r1 = total * (blockIdx.x + 1) / gridDim.x;
   if (r0 >= r1) return;
-  if (tid < 32) {
-    const int a = warp_slot_search(off, S, r0);
-    const int b = warp_slot_search(off, S, r1 - 1);
-    if (tid == 0) { s_first_sh = a; s_last_sh = b; }
+  if (!LAYOUT) {
+    if (tid < 32) {
+      const int a = warp_slot_search(off, S, r0);
+      const int b = warp_slot_search(off, S, r1 - 1);
+      if (tid == 0) { s_first_sh = a; s_last_sh = b; }
+    }
+    __syncthreads();
+    s_first = s_first_sh;
+    ns = s_last_sh - s_first_sh + 1;
+    staged = ns <= CP_MAX_SLOTS;
+    if (staged) {
+      for (int i = tid; i <= ns; i += blockDim.x) s_off[i] = off[s_first + i];
+      for (int i = tid; i < ns; i += blockDim.x) s_cnt[i] = min(count[s_first + i], max_sel);
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  const int s_first = s_first_sh, ns = s_last_sh - s_first_sh + 1;
-  const bool staged = ns <= CP_MAX_SLOTS;
-  if (staged) {
-    for (int i = tid; i <= ns; i += blockDim.x) s_off[i] = off[s_first + i];
-    for (int i = tid; i < ns; i += blockDim.x) s_cnt[i] = min(count[s_first + i], max_sel);
-  }
-  __syncthreads();
   constexpr int GROUPS = CP_THREADS / TPR;
   const int part = tid % TPR, grp = tid / TPR;
   for (long long base = r0; base < r1; base += CP_THREADS) {

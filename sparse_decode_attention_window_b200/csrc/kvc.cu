@@ -767,35 +767,51 @@ kvc_status kvc_layout(const int32_t* count, int32_t n_slots, int32_t reserve, in
   return check_launch("kvc_layout");
 }
 
-kvc_status kvc_compact(const kvc_shape* shape, const void* k, const void* v, const int32_t* idx, int32_t max_sel,
-                       const int32_t* count, const int64_t* off, void* kp, void* vp, int64_t kp_rows, int32_t* len,
-                       cudaStream_t stream) {
+// Compaction, after the layout (off given) or, with `layout`, computing it in the same launch
+// (off_out and cap_out written; S <= CP_MAX_SLOTS on the one-wave kernel).
+static kvc_status launch_compact(const char* what, const kvc_shape* shape, const void* k, const void* v,
+                                 const int32_t* idx, int32_t max_sel, const int32_t* count, const int64_t* off,
+                                 void* kp, void* vp, int64_t kp_rows, int32_t* len, bool layout, int32_t reserve,
+                                 int64_t* off_out, int32_t* cap_out, cudaStream_t stream) {
   kvc_status rc = check_shape(shape, false);
   if (rc != KVC_OK) return rc;
-  if (!k || !v || !idx || !count || !off || !kp || !vp || !len)
-    return fail(KVC_ERR_INVALID_ARG, "kvc_compact: NULL pointer argument");
-  if (max_sel <= 0 || kp_rows < 0) return fail(KVC_ERR_SHAPE, "kvc_compact: max_sel > 0, kp_rows >= 0 required");
+  if (!k || !v || !idx || !count || !(layout ? off_out && cap_out : off != nullptr) || !kp || !vp || !len)
+    return fail(KVC_ERR_INVALID_ARG, "%s: NULL pointer argument", what);
+  if (max_sel <= 0 || kp_rows < 0) return fail(KVC_ERR_SHAPE, "%s: max_sel > 0, kp_rows >= 0 required", what);
+  if (layout && reserve < 0) return fail(KVC_ERR_SHAPE, "%s: reserve >= 0 required", what);
   if (!aligned16(k) || !aligned16(v) || !aligned16(kp) || !aligned16(vp))
-    return fail(KVC_ERR_INVALID_ARG, "kvc_compact: k, v, kp, vp must be 16-byte aligned");
+    return fail(KVC_ERR_INVALID_ARG, "%s: k, v, kp, vp must be 16-byte aligned", what);
   DevInfo* di = nullptr;
   if ((rc = dev_info(&di)) != KVC_OK) return rc;
   const int tpr = (int)(shape->d * esize(shape->dtype) / 16);
+  if (tpr != 8 && tpr != 16 && tpr != 32) return fail(KVC_ERR_UNSUPPORTED, "%s: row of %d bytes", what, tpr * 16);
   const uint4* k4 = static_cast<const uint4*>(k);
   const uint4* v4 = static_cast<const uint4*>(v);
   uint4* kp4 = static_cast<uint4*>(kp);
   uint4* vp4 = static_cast<uint4*>(vp);
   const int S = shape->n_slots, L = shape->L;
+  if (layout && (S > kvc::CP_MAX_SLOTS || force_old_compact())) {
+    // more slots than one CTA stages: the layout kernel first, then the plain compaction
+    if ((rc = kvc_layout(count, S, reserve, off_out, cap_out, stream)) != KVC_OK) return rc;
+    return launch_compact(what, shape, k, v, idx, max_sel, count, off_out, kp, vp, kp_rows, len, false, 0, nullptr,
+                          nullptr, stream);
+  }
   if (!force_old_compact()) {
     const int blocks = di->sms * 4;   // one wave at four CTAs per SM
-    switch (tpr) {
-      case 8: kvc::compact_wave_kernel<8><<<blocks, kvc::CP_THREADS, 0, stream>>>(k4, v4, idx, max_sel, count, off, S,
-                                                                                  L, kp4, vp4, kp_rows, len); break;
-      case 16: kvc::compact_wave_kernel<16><<<blocks, kvc::CP_THREADS, 0, stream>>>(k4, v4, idx, max_sel, count, off,
-                                                                                    S, L, kp4, vp4, kp_rows, len); break;
-      case 32: kvc::compact_wave_kernel<32><<<blocks, kvc::CP_THREADS, 0, stream>>>(k4, v4, idx, max_sel, count, off,
-                                                                                    S, L, kp4, vp4, kp_rows, len); break;
-      default: return fail(KVC_ERR_UNSUPPORTED, "kvc_compact: row of %d bytes", tpr * 16);
+#define KVC_COMPACT_WAVE(T, LY)                                                                                  \
+  kvc::compact_wave_kernel<T, LY><<<blocks, kvc::CP_THREADS, 0, stream>>>(k4, v4, idx, max_sel, count, off, S, L, \
+                                                                          kp4, vp4, kp_rows, len, reserve, off_out, \
+                                                                          cap_out)
+    if (layout) {
+      if (tpr == 8) KVC_COMPACT_WAVE(8, true);
+      else if (tpr == 16) KVC_COMPACT_WAVE(16, true);
+      else KVC_COMPACT_WAVE(32, true);
+    } else {
+      if (tpr == 8) KVC_COMPACT_WAVE(8, false);
+      else if (tpr == 16) KVC_COMPACT_WAVE(16, false);
+      else KVC_COMPACT_WAVE(32, false);
     }
+#undef KVC_COMPACT_WAVE
   } else {
     const int blocks = di->sms * 8;
     switch (tpr) {
@@ -803,13 +819,26 @@ kvc_status kvc_compact(const kvc_shape* shape, const void* k, const void* v, con
                                                                      kp_rows, len); break;
       case 16: kvc::compact_kernel<16, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, S, L, kp4,
                                                                        vp4, kp_rows, len); break;
-      case 32: kvc::compact_kernel<32, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, S, L, kp4,
+      default: kvc::compact_kernel<32, 4><<<blocks, 256, 0, stream>>>(k4, v4, idx, max_sel, count, off, S, L, kp4,
                                                                        vp4, kp_rows, len); break;
-      default: return fail(KVC_ERR_UNSUPPORTED, "kvc_compact: row of %d bytes", tpr * 16);
     }
   }
   count_launches(1);
-  return check_launch("kvc_compact");
+  return check_launch(what);
+}
+
+kvc_status kvc_compact(const kvc_shape* shape, const void* k, const void* v, const int32_t* idx, int32_t max_sel,
+                       const int32_t* count, const int64_t* off, void* kp, void* vp, int64_t kp_rows, int32_t* len,
+                       cudaStream_t stream) {
+  return launch_compact("kvc_compact", shape, k, v, idx, max_sel, count, off, kp, vp, kp_rows, len, false, 0, nullptr,
+                        nullptr, stream);
+}
+
+kvc_status kvc_layout_compact(const kvc_shape* shape, const void* k, const void* v, const int32_t* idx,
+                              int32_t max_sel, const int32_t* count, int32_t reserve, int64_t* off, int32_t* cap,
+                              void* kp, void* vp, int64_t kp_rows, int32_t* len, cudaStream_t stream) {
+  return launch_compact("kvc_layout_compact", shape, k, v, idx, max_sel, count, nullptr, kp, vp, kp_rows, len, true,
+                        reserve, off, cap, stream);
 }
 
 kvc_status kvc_append_window(const kvc_shape* shape, const void* k_new, const void* v_new, const int64_t* off,

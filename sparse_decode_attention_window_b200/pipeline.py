@@ -15,7 +15,7 @@ import torch
 
 import math
 
-from . import (kvc_score, kvc_select, kvc_alloc_budgets, kvc_layout, kvc_compact, kvc_append, kvc_decode_attn,
+from . import (kvc_score, kvc_select, kvc_alloc_budgets, kvc_layout_compact, kvc_append, kvc_decode_attn,
                kvc_append_decode, kvc_append_decode_chain, kvc_select_chunks, kvc_append_window, KVC_POL_LOCAL,
                kvc_workspace_size, make_shape, KVC_WS_SCORE, KVC_WS_DECODE, KVC_POL_TOPB, KVC_POL_MASS_COUNT,
                KVC_POL_CHUNK)
@@ -158,9 +158,8 @@ class KvcPipeline:
             self.len_f.fill_(self.wl.L)    # the full cache restarts from the prompt
         if self.sliding:
             self.head.zero_()              # compaction stores a local head's window oldest first
-        kvc_layout(self.count, self.wl.reserve, self.off, self.cap, stream=stream)
-        kvc_compact(self.shape, self.inp.k, self.inp.v, self.idx, self.count, self.off, self.kp, self.vp, self.len,
-                    stream=stream)
+        kvc_layout_compact(self.shape, self.inp.k, self.inp.v, self.idx, self.count, self.wl.reserve, self.off,
+                           self.cap, self.kp, self.vp, self.len, stream=stream)
         self._chained = False              # the next decode follows a kernel that wrote the kept rows
 
     def compress(self, stream=None):
@@ -216,9 +215,8 @@ class KvcPipeline:
         shape_n = make_shape(S, G, d, n, 1, wl.hkv, wl.batch, self.kf.dtype)   # n tokens to choose from
         kvc_select_chunks(shape_n, score, ends, self.targets[i], self.idx, self.count, n_local=wl.n_local,
                           stream=stream)
-        kvc_layout(self.count, wl.steps - t - 1, self.off, self.cap, stream=stream)
-        kvc_compact(self.shape_full, self.kf, self.vf, self.idx, self.count, self.off, self.kp, self.vp, self.len,
-                    stream=stream)
+        kvc_layout_compact(self.shape_full, self.kf, self.vf, self.idx, self.count, wl.steps - t - 1, self.off,
+                           self.cap, self.kp, self.vp, self.len, stream=stream)
         self._chained = False
 
     def run(self, steps=None, record=False, stream=None):

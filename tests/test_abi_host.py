@@ -83,6 +83,19 @@ def test_layout_and_append_validate():
     assert lib.kvc_append(ctypes.byref(_shape()), misaligned, p, p, p, p, p, p, 64, None) == _abi.KVC_ERR_INVALID_ARG
 
 
+def test_layout_compact_validates():
+    lib = kvc.library()
+    p = ctypes.c_void_p(16)
+    sh = ctypes.byref(_shape())
+    f = lib.kvc_layout_compact
+    assert f(sh, p, p, p, 64, p, 4, None, p, p, p, 1024, p, None) == _abi.KVC_ERR_INVALID_ARG   # no off
+    assert f(sh, p, p, p, 64, p, 4, p, None, p, p, 1024, p, None) == _abi.KVC_ERR_INVALID_ARG   # no cap
+    assert f(sh, p, p, p, 64, p, -1, p, p, p, p, 1024, p, None) == _abi.KVC_ERR_SHAPE           # reserve < 0
+    assert f(sh, p, p, p, 0, p, 4, p, p, p, p, 1024, p, None) == _abi.KVC_ERR_SHAPE             # max_sel 0
+    assert f(sh, p, ctypes.c_void_p(24), p, 64, p, 4, p, p, p, p, 1024, p, None) == _abi.KVC_ERR_INVALID_ARG
+    assert b"kvc_layout_compact" in lib.kvc_last_error()
+
+
 def test_select_validates_mass_and_chunks():
     lib = kvc.library()
     p = ctypes.c_void_p(16)

@@ -670,6 +670,51 @@ def test_chained_append_decode_reports_a_broken_promise():
     kvc.kvc_get_status()
 
 
+@pytest.mark.parametrize("S,d,dt", [(4, 128, torch.bfloat16), (37, 64, torch.bfloat16), (512, 128, torch.bfloat16),
+                                    (600, 64, torch.bfloat16), (24, 128, torch.float32)])
+def test_layout_compact_matches_the_two_calls(S, d, dt):
+    """One launch of layout + compaction (or, above 512 slots, the two launches it falls back
+    to) gives the same offsets, capacities, lengths and packed rows, byte for byte, as
+    kvc_layout then kvc_compact; counts are ragged, with empty and negative slots and counts
+    above max_sel."""
+    import sparse_decode_attention_window_b200 as kvc
+    L, max_sel, reserve = 300, 160, 5
+    g = torch.Generator().manual_seed(S * 7 + d)
+    count = torch.randint(0, max_sel + 1, (S,), generator=g, dtype=torch.int32)
+    count[0] = 0
+    count[min(1, S - 1)] = max_sel
+    if S > 2:
+        count[2] = -3
+    if S > 3:
+        count[3] = max_sel + 40                # more than idx holds: max_sel rows copied
+    idx = torch.stack([torch.sort(torch.randperm(L, generator=g)[:max_sel])[0] for _ in range(S)]).to(torch.int32)
+    k = torch.randn((S, L, d), generator=g).to(dt).cuda()
+    v = torch.randn((S, L, d), generator=g).to(dt).cuda()
+    sh = kvc.make_shape(S, 1, d, L, 0, S, 1, dt)
+    rows = int(sum((max(int(c), 0) + reserve + 15) // 16 * 16 for c in count))
+    cnt, ix = count.cuda(), idx.cuda()
+    outs = []
+    for fused in (True, False):
+        off = torch.full((S + 1,), -7, dtype=torch.int64, device="cuda")
+        cap = torch.full((S,), -7, dtype=torch.int32, device="cuda")
+        ln = torch.full((S,), -7, dtype=torch.int32, device="cuda")
+        kp = torch.zeros((rows, d), dtype=dt, device="cuda")
+        vp = torch.zeros((rows, d), dtype=dt, device="cuda")
+        if fused:
+            kvc.kvc_layout_compact(sh, k, v, ix, cnt, reserve, off, cap, kp, vp, ln)
+        else:
+            kvc.kvc_layout(cnt, reserve, off, cap)
+            kvc.kvc_compact(sh, k, v, ix, cnt, off, kp, vp, ln)
+        kvc.kvc_get_status()
+        outs.append([off.cpu(), cap.cpu(), ln.cpu(), kp.view(torch.uint8).cpu(), vp.view(torch.uint8).cpu()])
+    for a, b, name in zip(outs[0], outs[1], ["off", "cap", "len", "kp", "vp"]):
+        assert torch.equal(a, b), name
+    # and the layout itself, by its definition
+    caps = [(max(int(c), 0) + reserve + 15) // 16 * 16 for c in count]
+    assert outs[0][1].tolist() == caps
+    assert outs[0][0].tolist() == [0] + list(np.cumsum(caps))
+
+
 def test_grid_stride_compaction_on_workloads():
     """The grid-stride compaction kernel (forced here; the one-wave kernel is the default)
     gives the same bit-exact packed caches."""
