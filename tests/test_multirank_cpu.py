@@ -53,9 +53,9 @@ def test_sharded_zigzag_allocation_matches_single_process():
     ref = O.allocate_budgets(np.array(counts).reshape(wl.n_layers, wl.slots_per_layer), wl.L, wl.avg_budget,
                              wl.floor_budget)
     world = 2
-    mgr = mp.Manager()
-    ret = mgr.dict()
     ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()               # its server process is spawned too: nothing forks
+    ret = mgr.dict()
     port = _free_port()
     procs = [ctx.Process(target=_worker, args=(r, world, port, counts, wl.n_layers, wl.slots_per_layer, wl.L,
                                                wl.avg_budget, wl.floor_budget, ret)) for r in range(world)]
