@@ -738,13 +738,6 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
         if (lane == 0) mbar_arrive(&empty[stage]);
         if (++stage == nst) { stage = 0; ph ^= 1; }
       }
-      // the two groups wait on different barriers: agree on an abort before any barrier
-      // that needs both of them
-      if (named_bar_or(1, C::CONS_THREADS, aborted)) {
-        aborted = true;
-        break;
-      }
-
       // ---- the warp's totals: l over its 8 row groups; PACK adds the remainder columns
 #pragma unroll
       for (int o_ = 4; o_ < 32; o_ <<= 1) {
@@ -757,38 +750,37 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
 #pragma unroll
           for (int j = 0; j < 4; ++j) o[dt][j] += __shfl_down_sync(0xffffffffu, o[dt][j], 2, 4);
       }
-      // ---- combine the 4 warps: common maximum per head, scaled sums
+      // ---- the warp's partial, unscaled (its own maximum m, sum l and output O); the combine
+      // below rescales each to the heads' common maximum
       if (g == 0) {
-        if (hv0) wm[cw * 8 + hc0] = m0;
-        if (hv1) wm[cw * 8 + hc1] = m1;
+        if (hv0) {
+          wm[cw * 8 + hc0] = m0;
+          wl[cw * 8 + hc0] = l0;
+        }
+        if (hv1) {
+          wm[cw * 8 + hc1] = m1;
+          wl[cw * 8 + hc1] = l1;
+        }
       }
-      named_bar_sync(1, C::CONS_THREADS);
-      float M0 = -INFINITY, M1 = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < C::CONS_WARPS; ++w) {
-        if (hv0) M0 = fmaxf(M0, wm[w * 8 + hc0]);
-        if (hv1) M1 = fmaxf(M1, wm[w * 8 + hc1]);
-      }
-      const float f0 = m0 == -INFINITY ? 0.f : ex2_ftz(m0 - M0);
-      const float f1 = m1 == -INFINITY ? 0.f : ex2_ftz(m1 - M1);
       float* wow = wo + (size_t)cw * G * C::WO_STRIDE;
 #pragma unroll
       for (int dt = 0; dt < C::DTILES; ++dt) {
         const int d0 = dt * 16 + g;
         if (hv0) {
-          wow[hc0 * C::WO_STRIDE + d0] = o[dt][0] * f0;
-          wow[hc0 * C::WO_STRIDE + d0 + 8] = o[dt][2] * f0;
+          wow[hc0 * C::WO_STRIDE + d0] = o[dt][0];
+          wow[hc0 * C::WO_STRIDE + d0 + 8] = o[dt][2];
         }
         if (hv1) {
-          wow[hc1 * C::WO_STRIDE + d0] = o[dt][1] * f1;
-          wow[hc1 * C::WO_STRIDE + d0 + 8] = o[dt][3] * f1;
+          wow[hc1 * C::WO_STRIDE + d0] = o[dt][1];
+          wow[hc1 * C::WO_STRIDE + d0 + 8] = o[dt][3];
         }
       }
-      if (g == 0) {
-        if (hv0) wl[cw * 8 + hc0] = l0 * f0;
-        if (hv1) wl[cw * 8 + hc1] = l1 * f1;
+      // one barrier for both: the partials are visible to every consumer thread, and the two
+      // groups (which wait on different stage barriers) agree on an abort
+      if (named_bar_or(1, C::CONS_THREADS, aborted)) {
+        aborted = true;
+        break;
       }
-      named_bar_sync(1, C::CONS_THREADS);
 
       const int cfirst = per_slot ? 0 : cta_of(P[s], s), clast = per_slot ? 0 : cta_of(P[s + 1] - 1, s);
       const bool single = !per_slot && cfirst == clast;
@@ -808,12 +800,17 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap mk64, const __grid_constan
       }
       for (int e = tid; e < G * D; e += C::CONS_THREADS) {
         const int h = e / D, d = e - h * D;
-        float A = 0.f, Mh = -INFINITY, Lh = 0.f;
+        float Mh = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < C::CONS_WARPS; ++w) Mh = fmaxf(Mh, wm[w * 8 + h]);
+        // each warp's share scaled by 2^(m_w - M): rounded products, then a sum in warp order
+        float A = 0.f, Lh = 0.f;
 #pragma unroll
         for (int w = 0; w < C::CONS_WARPS; ++w) {
-          A += wo[((size_t)w * G + h) * C::WO_STRIDE + d];
-          Mh = fmaxf(Mh, wm[w * 8 + h]);
-          Lh += wl[w * 8 + h];
+          const float mw = wm[w * 8 + h];
+          const float f = mw == -INFINITY ? 0.f : ex2_ftz(mw - Mh);
+          A += __fmul_rn(wo[((size_t)w * G + h) * C::WO_STRIDE + d], f);
+          Lh += __fmul_rn(wl[w * 8 + h], f);
         }
         if (per_slot && my_rank == 0) {
           rec[e] = A;
