@@ -37,7 +37,7 @@ UNIT = "tokens/s"
 # DRAM bytes (read + written) per launch of the decode kernel from one ncu capture of the
 # current kernel (cold-cache replay): llama8b 17.24 MB read + 0 written; zigzag cut to 8
 # layers 215.7 + 4.9 MB, scaled to the 32 layers (4x the cached rows, traffic in proportion).
-DECODE_TRAFFIC = {"llama8b": 17.17e6, "zigzag": 4 * (215.63e6 + 1.63e6)}
+DECODE_TRAFFIC = {"llama8b": 17.16e6, "zigzag": 4 * (215.63e6 + 1.78e6)}
 DECODE_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum of one capture of this kernel"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
