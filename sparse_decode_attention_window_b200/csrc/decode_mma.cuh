@@ -5,9 +5,16 @@
 // the compacted cache):
 //   out[h] = sum_{r < len[s]} softmax_r(q_h . K[off_s + r] / sqrt(d)) V[off_s + r].
 //
-// The work split and the merge are those of the CUDA-core decode (decode.cuh):
-// the valid tokens of all slots are cut into equal ranges, one per CTA, ranges may
-// cross slot boundaries, and the last CTA to finish a slot merges its partials.
+// Two work splits, chosen on the device from the plan lengths:
+//  - token ranges (as the CUDA-core decode, decode.cuh): the tokens of all slots are
+//    cut into ranges of equal cost, one per CTA, ranges may cross slot boundaries,
+//    and the last CTA to finish a slot merges the partials through global memory;
+//  - per-slot clusters, for few near-uniform slots: slot j gets cluster j of k CTAs,
+//    each sends its record (outputs, maxima, sums) into rank 0's shared memory by
+//    st.async and rank 0 merges them.
+// Inside a CTA, eight consumer warps (two groups of four, alternate 64-token tiles)
+// each keep an online-softmax partial; one barrier publishes the unscaled partials
+// and the combining threads rescale them to the common maximum.
 //
 // Why tensor cores here: the kernel is HBM-bound (4 flop per byte at G = 4), but
 // on the CUDA cores it needed ~67 warp instructions per cached token and stayed
