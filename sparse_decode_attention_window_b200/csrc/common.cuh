@@ -235,7 +235,7 @@ KVC_DEV void bulk_g2s(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t
       : "memory");
 }
 
-// Tiled TMA load of a 3-D box (no multicast). c0 is the innermost coordinate.
+// Tiled TMA load of a 3-D box into this CTA's shared memory. c0 is the innermost coordinate.
 KVC_DEV void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c0, int c1, int c2, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
