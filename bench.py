@@ -186,7 +186,7 @@ def reference_arm(args, wl, rank, world):
                    "l2": "n/a (host)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": f"each step: whole slots of the workload (score, select, all decode steps) "
-                                   f"for ~{args.ref_step_seconds:.0f} s, scaled to all {wl.n_slots} slots"},
+                                   f"for ~{args.ref_step_seconds:g} s, scaled to all {wl.n_slots} slots"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
