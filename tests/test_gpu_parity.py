@@ -773,6 +773,36 @@ def test_tcgen05_decode_path_on_bf16_workloads():
 
 
 # ---------------------------------------------------------------- next rows
+@pytest.mark.parametrize("dt,d,G,w,L", [("bf16", 128, 4, 32, 1000), ("bf16", 64, 2, 16, 777),
+                                        ("fp32", 128, 4, 8, 600)])
+def test_score_with_prefill_row_normalisers(dt, d, G, w, L):
+    """kvc_score given each window row's softmax normaliser from prefill (natural log over the
+    keys the row sees) skips its statistics pass; the scores still match the oracle's."""
+    import sparse_decode_attention_window_b200 as kvc
+    S = 6
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    g = torch.Generator().manual_seed(L + d)
+    q = torch.randn((S * G, w, d), generator=g).to(tdt)
+    k = torch.randn((S, L, d), generator=g).to(tdt)
+    # the caller's normalisers, in fp64 from the same rounded inputs (row i sees keys <= L - w + i)
+    qd, kd = q.double().numpy(), k.double().numpy()
+    lse = np.empty((S * G, w))
+    for s in range(S):
+        z = np.einsum("jid,nd->jin", qd[s * G:(s + 1) * G], kd[s]) / math.sqrt(d)
+        for i in range(w):
+            zi = z[:, i, :L - w + i + 1]
+            m = zi.max(axis=1)
+            lse[s * G:(s + 1) * G, i] = m + np.log(np.exp(zi - m[:, None]).sum(axis=1))
+    sh = kvc.make_shape(S, G, d, L, w, 1, S, tdt)
+    ws = torch.zeros(kvc.kvc_workspace_size(kvc.KVC_WS_SCORE, sh), dtype=torch.uint8, device="cuda")
+    score = torch.empty((S, L), device="cuda")
+    kvc.kvc_score(sh, q.cuda(), k.cuda(), score, ws,
+                  row_lse=torch.tensor(lse.reshape(-1), dtype=torch.float32, device="cuda"))
+    kvc.kvc_get_status()
+    ref = np.stack([O.window_scores(q[s * G:(s + 1) * G], k[s:s + 1], L)[0] for s in range(S)])
+    P.check_scores(_np(score), ref, dt, f"row_lse {dt} d{d} G{G} w{w} L{L}")
+
+
 def test_retained_mass_matches_oracle():
     """Attention retained by the selection (ZigZagKV's attention loss is 0.9 minus it)."""
     import sparse_decode_attention_window_b200 as kvc
