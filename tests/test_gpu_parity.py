@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle as O
-from workloads import get, make_inputs, POL_LOCAL, POL_SPECIAL, POL_FULL
+from workloads import get, make_inputs, POL_LOCAL, POL_SPECIAL
 from tests import parity as P
 
 pytestmark = pytest.mark.gpu

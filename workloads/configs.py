@@ -27,7 +27,7 @@ Nothing here computes any part of the method; this module only holds sizes.
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field, replace
+from dataclasses import dataclass, replace
 
 
 @dataclass(frozen=True)
