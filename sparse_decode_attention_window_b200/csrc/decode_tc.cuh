@@ -64,7 +64,7 @@ struct DtCfg {
 struct DtLayout {
   int nst;                                           // pipeline stages (2 or 3)
   size_t stages, pbuf, bars, P, offs, red, xr, app, total;
-  KVC_HD static DtLayout make(int S, int G, int grid, int ksz, int nst) {
+  KVC_HD static DtLayout make(int S, int G, int /* grid: unused, kept for the callers */, int ksz, int nst) {
     using C = DtCfg;
     DtLayout l{};
     l.nst = nst;
