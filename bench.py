@@ -5,7 +5,11 @@ One step = one pass of the whole path over one batch of synthetic input: score,
 select (and allocate), layout, compact, then `steps` decode steps (append +
 decode attention). Prints ONE JSON line on rank 0.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b] [--impl kvc|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload zigzag] [--impl kvc|reference]
+
+The default workload is ZigZagKV's: 32 layers of the LLaMA-3-8B attention shape at 32K
+context with per-layer budgets, the largest one that fits one GPU (its packed cache,
+~0.86 GB per decode step, does not fit in L2).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (weak
 scaling, no data-path collective); times are the max over ranks.
@@ -132,58 +136,170 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle timing (CPU baseline / reference arm)
-_ORACLE_INPUTS = {}
+def oracle_workload(wl):
+    """The workload the oracle is timed on: whole slots of the same shapes and per-slot work.
+    A many-layer workload is cut to its first layer (its slots have the layers' shapes; the
+    per-layer budgets are replaced by their average, which is what the slots keep on average)."""
+    return wl.scaled(n_layers=1) if wl.n_layers > 1 else wl
 
 
-def oracle_sample(wl, budget_s: float, seed_slots=0):
-    """Time the oracle on whole slots (scoring, selection, all decode steps) until `budget_s`
-    seconds pass or the workload is done; returns (seconds, slots done, threads)."""
-    from threadpoolctl import threadpool_limits
+_ORACLE = {}            # per process: the oracle workload's host inputs, by workload name
+
+
+def _oracle_inputs(wl):
+    if wl.name not in _ORACLE:
+        _ORACLE[wl.name] = make_inputs(wl, "cpu")
+    return _ORACLE[wl.name]
+
+
+def _oracle_slot(wl, inp, s):
+    """The oracle's whole pipeline for slot `s` of `wl`: scoring, selection and every decode step."""
     from oracle.pipeline import run_workload
-    if wl.name not in _ORACLE_INPUTS:
-        _ORACLE_INPUTS[wl.name] = make_inputs(wl, "cpu")
-    inp = _ORACLE_INPUTS[wl.name]
-    S = wl.n_slots
-    order = list(range(S))
-    rng = np.random.default_rng(seed_slots)
-    rng.shuffle(order)
-    with threadpool_limits(limits=1):
-        budgets = None
+    budgets = None
+    if wl.policy == "zigzag":
+        budgets = np.full(wl.n_layers, wl.avg_budget, dtype=np.int64)
+    run_workload(inp, slots=[s], budgets=budgets)
+
+
+def _pool_init(wl, inp):
+    # one thread per worker: the pool's processes are the parallelism
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(limits=1)
+    torch.set_num_threads(1)
+    _ORACLE["pool"] = (wl, inp)
+
+
+def _pool_ready(_):
+    time.sleep(0.05)
+    return os.getpid()
+
+
+def _pool_task(s):
+    wl, inp = _ORACLE["pool"]
+    _oracle_slot(wl, inp, s)
+    return s
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+class OracleTimer:
+    """Times the oracle on whole slots of `oracle_workload(wl)`: on one thread, and on every
+    host core as a pool of one-thread processes (started with spawn, each process receives
+    the inputs in shared memory)."""
+
+    def __init__(self, wl):
+        self.full = wl
+        self.wl = oracle_workload(wl)
+        self.inp = _oracle_inputs(self.wl)
+        self.pool = None
+        self.cores = 1
+
+    def one_core(self, budget_s: float, seed: int = 0):
+        """(seconds per slot, slots done, seconds) on one thread, whole slots until budget_s pass."""
+        from threadpoolctl import threadpool_limits
+        order = list(range(self.wl.n_slots))
+        np.random.default_rng(seed).shuffle(order)
+        nthr = torch.get_num_threads()
+        torch.set_num_threads(1)
+        try:
+            with threadpool_limits(limits=1):
+                t0 = time.perf_counter()
+                done = 0
+                while True:
+                    _oracle_slot(self.wl, self.inp, order[done % len(order)])
+                    done += 1
+                    if time.perf_counter() - t0 >= budget_s:
+                        break
+                dt = time.perf_counter() - t0
+        finally:
+            torch.set_num_threads(nthr)
+        return dt / done, done, dt
+
+    def start_pool(self, cores: int | None = None):
+        import torch.multiprocessing as tmp
+        self.cores = max(1, cores or host_cores())
+        for t in vars(self.inp).values():
+            if isinstance(t, torch.Tensor):
+                t.share_memory_()
+        ctx = tmp.get_context("spawn")
+        self.pool = ctx.Pool(self.cores, initializer=_pool_init, initargs=(self.wl, self.inp))
+        # every worker has initialised once each has taken one of these
+        self.pool.map(_pool_ready, range(2 * self.cores), chunksize=1)
+
+    def all_cores(self, n_slots: int, seed: int = 0):
+        """(seconds per slot, slots done, seconds) for n_slots whole slots over the pool."""
+        S = self.wl.n_slots
+        order = [int(x) for x in np.random.default_rng(seed).integers(0, S, size=n_slots)]
         t0 = time.perf_counter()
-        done = 0
-        for s in order:
-            if wl.policy == "zigzag":
-                # timing sample only: the allocation needs every slot's LMBA count, so the
-                # sampled slots keep the average budget
-                budgets = np.full(wl.n_layers, wl.avg_budget, dtype=np.int64)
-            run_workload(inp, slots=[s], budgets=budgets)
-            done += 1
-            if time.perf_counter() - t0 >= budget_s:
-                break
+        self.pool.map(_pool_task, order, chunksize=max(1, n_slots // (8 * self.cores)))
         dt = time.perf_counter() - t0
-    return dt, done, 1
+        return dt / n_slots, n_slots, dt
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.close()
+            self.pool.join()
+            self.pool = None
+
+
+def cpu_baseline_leg(wl, one_core_s: float, all_cores_s: float):
+    """The oracle's throughput in the bench's unit: all host cores (the headline) and one core."""
+    tm = OracleTimer(wl)
+    per1, done1, dt1 = tm.one_core(one_core_s)
+    tokens = wl.batch * wl.steps
+    full1 = per1 * wl.n_slots
+    one = {"value": tokens / full1, "unit": UNIT, "cores": 1,
+           "sample": f"{done1} whole slots (score, select, {wl.steps} decode steps each) in {dt1:.1f} s on one "
+                     f"thread, scaled to the step's {wl.n_slots} slots ({full1:.1f} s)"}
+    tm.start_pool()
+    try:
+        n = max(tm.cores, int(all_cores_s / per1 * tm.cores))
+        perN, doneN, dtN = tm.all_cores(n)
+    finally:
+        tm.close()
+    fullN = perN * wl.n_slots
+    sample_wl = tm.wl
+    cut = (f" of a {sample_wl.n_layers}-layer cut of the workload (budgets at their average)"
+           if sample_wl is not wl else "")
+    return {"value": tokens / fullN, "unit": UNIT, "cores": tm.cores, "kind": "oracle",
+            "sample": f"{doneN} whole slots{cut} (score, select, {wl.steps} decode steps each) in {dtN:.1f} s over "
+                      f"{tm.cores} one-thread processes, scaled to the step's {wl.n_slots} slots ({fullN:.2f} s)",
+            "one_core": one}
 
 
 def reference_arm(args, wl, rank, world):
     if rank != 0:
         return 0
     tokens = wl.batch * wl.steps
+    tm = OracleTimer(wl)
+    per1, _, _ = tm.one_core(min(args.ref_step_seconds, 2.0))
+    tm.start_pool()
     per_step = []
-    for i in range(args.warmup + args.steps):
-        dt, done, cores = oracle_sample(wl, args.ref_step_seconds, seed_slots=i)
-        if i >= args.warmup:
-            per_step.append(dt * wl.n_slots / done)
+    try:
+        n = max(tm.cores, int(args.ref_step_seconds / per1 * tm.cores))
+        for i in range(args.warmup + args.steps):
+            per, _, _ = tm.all_cores(n, seed=i)
+            if i >= args.warmup:
+                per_step.append(per * wl.n_slots)
+    finally:
+        tm.close()
     ms = 1000.0 * statistics.mean(per_step)
     value = tokens / (ms / 1000.0)
+    cut = (f" of a {tm.wl.n_layers}-layer cut of the workload (budgets at their average)" if tm.wl is not wl else "")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.batch, "context": wl.L, "decode_steps": wl.steps,
-                   "l2": "n/a (host)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"each step: whole slots of the workload (score, select, all decode steps) "
-                                   f"for ~{args.ref_step_seconds:g} s, scaled to all {wl.n_slots} slots"},
+                   "layers": wl.n_layers, "l2": "n/a (host)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": tm.cores, "kind": "oracle",
+                         "sample": f"each step: {n} whole slots{cut} (score, select, all decode steps) over "
+                                   f"{tm.cores} one-thread processes, scaled to the step's {wl.n_slots} slots"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -350,11 +466,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
     # ---- CPU baseline (rank 0, single GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, done, cores = oracle_sample(wl, args.cpu_seconds)
-        full = dt * wl.n_slots / done
-        cpu = {"value": wl.batch * wl.steps / full, "unit": UNIT, "cores": cores, "kind": "oracle",
-               "sample": f"{done} of {wl.n_slots} slots (score, select, {wl.steps} decode steps each) in "
-                         f"{dt:.1f} s on 1 thread, scaled to the whole step ({full:.1f} s)"}
+        cpu = cpu_baseline_leg(wl, args.cpu_seconds, args.cpu_seconds)
 
     del graph, graph_ph
     if world > 1:
@@ -410,7 +522,7 @@ def cuda_arm(args, wl, rank, world, local_rank):
         "timing": "each step is one CUDA-graph replay of the C-ABI calls, timed by external CUDA events "
                   "at its two ends; phase and per-launch times from a second graph of the same calls with "
                   "events between the phases (which stop launches overlapping there); decode per launch = "
-                  "the 64-launch loop time / launches",
+                  f"the {n_dec}-launch loop time / {n_dec}",
         "e2e": e2e,
         "warm_l2": {"ms_per_step": statistics.mean(warm_ms), "steps": len(warm_ms),
                     "note": "no L2 flush between steps (inputs partly L2-resident); not the metric"},
@@ -473,7 +585,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="llama8b")
+    ap.add_argument("--workload", default="zigzag")
     ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

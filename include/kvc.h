@@ -264,14 +264,21 @@ kvc_status kvc_append_decode_chain(const kvc_shape* shape, const void* k_new, co
  *   time, with no allocator and no workspace handle), or loops where a
  *   cudaMalloc's implicit device synchronisation is not acceptable. The paper has
  *   no counterpart; this is a property of the library, not of the method.
- *   Same arguments and results as kvc_decode_attn minus the workspace: the
- *   scratch lives in a fixed 4 MiB array inside the library (held by every GPU
- *   that loads it, until exit). The first call on each device looks up that
- *   array's device address (make it before any stream capture). Shapes whose
- *   scratch (kvc_workspace_size(KVC_WS_DECODE, ...)) exceeds 4 MiB are rejected
- *   with KVC_ERR_WORKSPACE. All calls share the array and each call clears the
- *   part that must start at zero: calls that overlap on the GPU (for example on
- *   two streams) race and must not be issued.
+ *   Same arguments as kvc_decode_attn minus the workspace: the scratch lives in a
+ *   fixed 4 MiB array inside the library (held by every GPU that loads it, until
+ *   exit). It always takes the token-range work split (the per-slot cluster form
+ *   kvc_decode_attn picks for few slots merges through shared memory, not the
+ *   scratch), so for shapes where kvc_decode_attn runs clusters the two sum the
+ *   partials in a different order: results agree within the decode tolerance, not
+ *   bit for bit. Scratch needed: 256-byte rounded (S + 1) * 4 B of tickets plus
+ *   (SMs + S) * round_up(G * (d + 2), 4) * 4 B of partials, 256-byte rounded
+ *   (= kvc_workspace_size(KVC_WS_DECODE, ...)); shapes needing more than 4 MiB are
+ *   rejected with KVC_ERR_WORKSPACE (G = 4, d = 128 on 148 SMs: up to 1864 slots).
+ *   The first successful call on each device looks up the array's device address
+ *   (make it before any stream capture); a failed lookup is retried on the next
+ *   call. All calls share the array and each call clears the part that must start
+ *   at zero: calls that overlap on the GPU (for example on two streams) race and
+ *   must not be issued.
  */
 kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const void* kp,
                                    const void* vp, const int64_t* off, const int32_t* len,
@@ -354,6 +361,38 @@ unsigned long long kvc_launch_count(void);
  *   KVC_ERR_INVALID_ARG.
  */
 kvc_status kvc_check_wait_limit(int32_t limit_us, cudaStream_t stream);
+
+/*
+ * kvc_diag_set_path - diagnostic, for cross-checks only: force one of the library's
+ *   alternate kernel paths for every later call in this process (all threads), so a
+ *   test can run the same inputs through both forms of a step and compare. Production
+ *   callers never call it: with every knob at 0 (the state at load) each call takes
+ *   the path its shape selects. Nothing else (no environment variable) changes a path.
+ *   knob (KVC_DIAG_*) and choice:
+ *     KVC_DIAG_SCORE        0 auto, 1 two-launch tensor-core form, 2 CUDA-core kernels
+ *     KVC_DIAG_SELECT       0 auto, 1 one CTA per slot
+ *     KVC_DIAG_COMPACT      0 auto, 1 grid-stride compaction kernel
+ *     KVC_DIAG_DECODE       0 auto, 1 CUDA-core decode, 2 tcgen05 decode (bf16, d = 128)
+ *     KVC_DIAG_DECODE_SPLIT 0 auto, 1 token-range split even for few slots
+ *   Unknown knob or choice: KVC_ERR_INVALID_ARG, nothing changed. Set it between calls,
+ *   not while another thread launches or a stream is being captured.
+ * kvc_diag_get_path - the current choice of `knob` (-1 for an unknown knob).
+ */
+#define KVC_DIAG_SCORE 0
+#define KVC_DIAG_SELECT 1
+#define KVC_DIAG_COMPACT 2
+#define KVC_DIAG_DECODE 3
+#define KVC_DIAG_DECODE_SPLIT 4
+#define KVC_DIAG_KNOBS 5
+#define KVC_DIAG_SCORE_TWO_PASS 1
+#define KVC_DIAG_SCORE_SIMT 2
+#define KVC_DIAG_SELECT_CTA 1
+#define KVC_DIAG_COMPACT_GRID 1
+#define KVC_DIAG_DECODE_SIMT 1
+#define KVC_DIAG_DECODE_TC 2
+#define KVC_DIAG_SPLIT_TOKENS 1
+kvc_status kvc_diag_set_path(int32_t knob, int32_t choice);
+int32_t kvc_diag_get_path(int32_t knob);
 
 #ifdef __cplusplus
 }

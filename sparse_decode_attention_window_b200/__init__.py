@@ -20,6 +20,7 @@ __all__ = ["KvcShape", "KvcError", "make_shape", "kvc_score", "kvc_select", "kvc
            "kvc_compact", "kvc_layout_compact", "kvc_append", "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_version",
            "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_append_decode_chain", "kvc_select_chunks",
            "kvc_retained_mass", "kvc_profile_heads", "kvc_append_window", "kvc_check_wait_limit",
+           "kvc_diag_set_path", "kvc_diag_get_path",
            "library", "KVC_BF16", "KVC_FP32", "KVC_POL_TOPB", "KVC_POL_MASS_COUNT", "KVC_POL_LOCAL",
            "KVC_POL_SPECIAL", "KVC_POL_FULL", "KVC_POL_CHUNK", "KVC_WS_SCORE", "KVC_WS_SELECT", "KVC_WS_DECODE"]
 
@@ -163,6 +164,19 @@ def kvc_check_wait_limit(limit_us, stream=None):
     """Diagnostic: a kernel waits on a barrier nothing arrives on until limit_us, gives up and
     flags a wait timeout (see include/kvc.h)."""
     _check("kvc_check_wait_limit", library().kvc_check_wait_limit(int(limit_us), _stream(stream)))
+
+
+def kvc_diag_set_path(knob: str, choice: str):
+    """Diagnostic, cross-checks only: force an alternate kernel path for every later call
+    in this process (knob, choice as in _abi.KVC_DIAG; "auto" restores the default)."""
+    k, choices = _abi.KVC_DIAG[knob]
+    _check("kvc_diag_set_path", library().kvc_diag_set_path(k, choices[choice]))
+
+
+def kvc_diag_get_path(knob: str) -> str:
+    k, choices = _abi.KVC_DIAG[knob]
+    v = int(library().kvc_diag_get_path(k))
+    return {c: n for n, c in choices.items()}[v]
 
 
 def kvc_get_status(stream=None):

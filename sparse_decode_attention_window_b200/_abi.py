@@ -24,7 +24,17 @@ EXPORTS = ["kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout", "kvc_co
            "kvc_append_window",
            "kvc_decode_attn", "kvc_workspace_size", "kvc_get_status", "kvc_last_error", "kvc_version",
            "kvc_launch_count", "kvc_decode_attn_noalloc", "kvc_append_decode", "kvc_append_decode_chain", "kvc_select_chunks",
-           "kvc_retained_mass", "kvc_profile_heads", "kvc_check_wait_limit"]
+           "kvc_retained_mass", "kvc_profile_heads", "kvc_check_wait_limit", "kvc_diag_set_path",
+           "kvc_diag_get_path"]
+
+# kvc_diag_set_path knobs and choices (cross-checks only)
+KVC_DIAG = {
+    "score": (0, {"auto": 0, "twopass": 1, "simt": 2}),
+    "select": (1, {"auto": 0, "cta": 1}),
+    "compact": (2, {"auto": 0, "grid": 1}),
+    "decode": (3, {"auto": 0, "simt": 1, "tc": 2}),
+    "decode_split": (4, {"auto": 0, "tokens": 1}),
+}
 
 
 class KvcShape(ctypes.Structure):
@@ -76,6 +86,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         "kvc_retained_mass": (i32, [sh, vp, i32, vp, i32, vp, vp, vp]),
         "kvc_profile_heads": (i32, [sh, vp, vp, i32, f32, vp, vp, vp]),
         "kvc_check_wait_limit": (i32, [i32, vp]),
+        "kvc_diag_set_path": (i32, [i32, i32]),
+        "kvc_diag_get_path": (i32, [i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

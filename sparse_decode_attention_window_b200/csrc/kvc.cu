@@ -108,63 +108,27 @@ kvc_status check_shape(const kvc_shape* sh, bool need_window) {
   return KVC_OK;
 }
 
-// KVC_SCORE_PATH=simt routes bf16 scoring to the CUDA-core kernels (used to cross-check
-// the two paths against each other); read once per process.
-bool force_simt() {
-  static const bool v = [] {
-    const char* e = getenv("KVC_SCORE_PATH");
-    return e && strcmp(e, "simt") == 0;
-  }();
-  return v;
-}
+// Kernel-path overrides for cross-checks, set only through kvc_diag_set_path (process-wide;
+// all zero = the automatic choice every production call makes). Nothing else changes them.
+std::atomic<int> g_diag[KVC_DIAG_KNOBS];
 
-// KVC_SCORE_PATH=twopass keeps tensor-core scoring in its two-launch form (pass 1, merge,
-// pass 2) where the fused slot-cluster kernel would run (cross-checks); read once.
-bool force_two_pass_score() {
-  static const bool v = [] {
-    const char* e = getenv("KVC_SCORE_PATH");
-    return e && strcmp(e, "twopass") == 0;
-  }();
-  return v;
-}
+int diag(int knob) { return g_diag[knob].load(std::memory_order_relaxed); }
 
-// KVC_SELECT_PATH=cta keeps selection at one CTA per slot (cross-checks); read once.
-bool force_cta_select() {
-  static const bool v = [] {
-    const char* e = getenv("KVC_SELECT_PATH");
-    return e && strcmp(e, "cta") == 0;
-  }();
-  return v;
-}
-
-// KVC_COMPACT_PATH=grid keeps the grid-stride compaction kernel (cross-checks); read once.
-bool force_old_compact() {
-  static const bool v = [] {
-    const char* e = getenv("KVC_COMPACT_PATH");
-    return e && strcmp(e, "grid") == 0;
-  }();
-  return v;
-}
-
-// KVC_DECODE_PATH=simt routes bf16 decode to the CUDA-core kernel (cross-checks); read once.
-bool force_simt_decode() {
-  static const bool v = [] {
-    const char* e = getenv("KVC_DECODE_PATH");
-    return e && strcmp(e, "simt") == 0;
-  }();
-  return v;
-}
-
-// KVC_DECODE_PATH=tc routes bf16, d = 128 decode to the tcgen05 kernel (decode_tc.cuh,
-// a cross-check and measurement path: on B200 it is slower than the mma.sync kernel, see
-// that file's header); read once.
-bool force_tc_decode() {
-  static const bool v = [] {
-    const char* e = getenv("KVC_DECODE_PATH");
-    return e && strcmp(e, "tc") == 0;
-  }();
-  return v;
-}
+// bf16 scoring on the CUDA-core kernels
+bool force_simt() { return diag(KVC_DIAG_SCORE) == KVC_DIAG_SCORE_SIMT; }
+// tensor-core scoring in its two-launch form where the fused slot-cluster kernel would run
+bool force_two_pass_score() { return diag(KVC_DIAG_SCORE) == KVC_DIAG_SCORE_TWO_PASS; }
+// selection at one CTA per slot where slot clusters would run
+bool force_cta_select() { return diag(KVC_DIAG_SELECT) == KVC_DIAG_SELECT_CTA; }
+// the grid-stride compaction kernel instead of the one-wave kernel
+bool force_old_compact() { return diag(KVC_DIAG_COMPACT) == KVC_DIAG_COMPACT_GRID; }
+// bf16 decode on the CUDA-core kernel
+bool force_simt_decode() { return diag(KVC_DIAG_DECODE) == KVC_DIAG_DECODE_SIMT; }
+// bf16, d = 128 decode on the tcgen05 kernel (decode_tc.cuh: slower than the mma.sync
+// kernel on B200, kept as a cross-check and measurement path)
+bool force_tc_decode() { return diag(KVC_DIAG_DECODE) == KVC_DIAG_DECODE_TC; }
+// the token-range decode split even for few slots
+bool force_token_split() { return diag(KVC_DIAG_DECODE_SPLIT) == KVC_DIAG_SPLIT_TOKENS; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -224,15 +188,6 @@ kvc_status launch_decode(const kvc::DecodeParams& p, int sms, cudaStream_t st) {
   decode_kernel<T, D, G><<<sms, DecCfg<T, D, G>::THREADS, smem, st>>>(p);
   count_launches(1);
   return check_launch("kvc_decode_attn");
-}
-
-// KVC_DECODE_SPLIT=tokens keeps the token-range split even for few slots (cross-checks).
-bool force_token_split() {
-  static const bool v = [] {
-    const char* e = getenv("KVC_DECODE_SPLIT");
-    return e && strcmp(e, "tokens") == 0;
-  }();
-  return v;
 }
 
 // How many clusters of k decode CTAs can be resident at once (shared memory per SM, GPC
@@ -473,24 +428,26 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[KVC_NOALLOC_SCR
 
 namespace {
 void* g_noalloc_ptr[kMaxDevices];
-cudaError_t g_noalloc_rc[kMaxDevices];
-std::once_flag g_noalloc_once[kMaxDevices];
+std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on the current device, looked up once per
-// device (the first call on a device does this; make that call before any stream
-// capture, since the lookup may load the module).
+// Device address of the scratch array on the current device, looked up by the first
+// successful call on that device (make it before any stream capture, since the lookup
+// may load the module); a failed lookup is not kept, the next call tries again.
 kvc_status noalloc_scratch(unsigned char** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(KVC_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(KVC_ERR_UNSUPPORTED, "device index %d out of range", dev);
-  std::call_once(g_noalloc_once[dev], [dev] {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
     void* p = nullptr;
-    g_noalloc_rc[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      cudaGetLastError();   // not sticky: leave no error for the next check
+      return fail(KVC_ERR_CUDA, "scratch address on device %d: %s", dev, cudaGetErrorString(e));
+    }
     g_noalloc_ptr[dev] = p;
-  });
-  if (g_noalloc_rc[dev] != cudaSuccess || !g_noalloc_ptr[dev])
-    return fail(KVC_ERR_CUDA, "scratch address on device %d: %s", dev, cudaGetErrorString(g_noalloc_rc[dev]));
+  }
   *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
   return KVC_OK;
 }
@@ -738,6 +695,22 @@ __global__ void wait_limit_probe_kernel(unsigned long long limit_ns) {
 }
 }  // namespace kvc
 
+kvc_status kvc_diag_set_path(int32_t knob, int32_t choice) {
+  static const int n_choices[KVC_DIAG_KNOBS] = {3, 2, 2, 3, 2};
+  if (knob < 0 || knob >= KVC_DIAG_KNOBS) return fail(KVC_ERR_INVALID_ARG, "kvc_diag_set_path: unknown knob %d", knob);
+  if (choice < 0 || choice >= n_choices[knob])
+    return fail(KVC_ERR_INVALID_ARG, "kvc_diag_set_path: choice %d not in [0, %d) for knob %d", choice,
+                n_choices[knob], knob);
+  g_diag[knob].store(choice, std::memory_order_relaxed);
+  g_last_error.clear();
+  return KVC_OK;
+}
+
+int32_t kvc_diag_get_path(int32_t knob) {
+  if (knob < 0 || knob >= KVC_DIAG_KNOBS) return -1;
+  return diag(knob);
+}
+
 kvc_status kvc_check_wait_limit(int32_t limit_us, cudaStream_t stream) {
   if (limit_us < 1 || limit_us > 1000000)
     return fail(KVC_ERR_INVALID_ARG, "kvc_check_wait_limit: limit_us = %d not in [1, 1e6]", limit_us);
@@ -906,8 +879,9 @@ kvc_status kvc_decode_attn(const kvc_shape* shape, const void* q, const void* kp
   return launch_decode_any(shape, p, di->sms, stream);
 }
 
-// Decode attention without a caller workspace: same kernel and results as
-// kvc_decode_attn, with its scratch in the fixed array above. Allocates nothing.
+// Decode attention without a caller workspace: the kvc_decode_attn kernel in its
+// token-range split (whose merge goes through the scratch), with the scratch in the
+// fixed array above. Allocates nothing.
 kvc_status kvc_decode_attn_noalloc(const kvc_shape* shape, const void* q, const void* kp, const void* vp,
                                    const int64_t* off, const int32_t* len, int64_t kp_rows, float* out,
                                    cudaStream_t stream) {

@@ -134,3 +134,36 @@ def test_fused_decode_entries_validate():
     bad = ctypes.byref(_shape(d=96))
     assert lib.kvc_append_decode_chain(bad, p, p, p, p, p, p, p, p, p, 64, p, p, 1 << 20, None) == \
         _abi.KVC_ERR_UNSUPPORTED
+
+
+def test_diagnostic_path_knobs_set_get_and_reject():
+    """Alternate kernel paths are chosen only through kvc_diag_set_path: every knob starts at
+    auto, takes its documented choices, rejects unknown knobs and choices, and returns to auto."""
+    lib = kvc.library()
+    for knob, (k, choices) in _abi.KVC_DIAG.items():
+        assert lib.kvc_diag_get_path(k) == 0, knob
+        for name, c in choices.items():
+            assert lib.kvc_diag_set_path(k, c) == _abi.KVC_OK
+            assert kvc.kvc_diag_get_path(knob) == name
+        assert lib.kvc_diag_set_path(k, len(choices)) == _abi.KVC_ERR_INVALID_ARG
+        assert lib.kvc_diag_set_path(k, -1) == _abi.KVC_ERR_INVALID_ARG
+        kvc.kvc_diag_set_path(knob, "auto")
+        assert lib.kvc_diag_get_path(k) == 0
+    assert lib.kvc_diag_set_path(len(_abi.KVC_DIAG), 0) == _abi.KVC_ERR_INVALID_ARG
+    assert lib.kvc_diag_get_path(len(_abi.KVC_DIAG)) == -1
+
+
+def test_environment_does_not_switch_kernel_paths():
+    """No environment variable reaches the library's path choice: a process started with the
+    old switch names set still reports every knob at auto."""
+    import subprocess
+    import sys
+    env = dict(os.environ, KVC_SCORE_PATH="simt", KVC_SELECT_PATH="cta", KVC_COMPACT_PATH="grid",
+               KVC_DECODE_PATH="tc", KVC_DECODE_SPLIT="tokens")
+    code = ("import sys; sys.path.insert(0, %r); import sparse_decode_attention_window_b200 as k; "
+            "print([k.library().kvc_diag_get_path(i) for i in range(5)])" % ROOT)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip().splitlines()[-1] == "[0, 0, 0, 0, 0]"
+    src = open(os.path.join(ROOT, "sparse_decode_attention_window_b200", "csrc", "kvc.cu")).read()
+    assert "getenv" not in src

@@ -3,7 +3,9 @@
 Small workloads are checked on every slot and step; the full-size workloads run
 in the same launch configuration the benchmark times and are checked on sampled
 slots and steps (the oracle computes them one by one)."""
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -352,15 +354,14 @@ def test_bounded_wait_gives_up_and_leaves_the_context_usable():
 def test_one_cta_per_slot_selection_on_workloads():
     """Selection at one CTA per slot (forced here; few slots take thread-block clusters by
     default) passes the same oracle checks."""
-    import os
     import subprocess
     import sys
-    env = dict(os.environ, KVC_SELECT_PATH="cta")
-    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+    forced = ['--kvc-path', 'select=cta']
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider", *forced,
                         "-k", "selection_policies_over_slot_counts or chunk_selection_over_slot_counts or "
                               "llama8b_shape_small_context or zigzag_small or chunk_small or budget_extremes or "
                               "mass_count_closed_forms or chunk_selection_with_local_chunks"],
-                       env=env, capture_output=True, text=True, timeout=900)
+                       capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
@@ -532,14 +533,13 @@ def test_wide_window_takes_cuda_core_scoring_path():
 
 def test_cuda_core_paths_on_bf16_workloads():
     """The CUDA-core scoring and decode kernels, forced for bf16, pass the same oracle checks."""
-    import os
     import subprocess
     import sys
-    env = dict(os.environ, KVC_SCORE_PATH="simt", KVC_DECODE_PATH="simt")
-    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+    forced = ['--kvc-path', 'score=simt', '--kvc-path', 'decode=simt']
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider", *forced,
                         "-k", "llama8b_shape_small_context or zigzag_small or chunk_small or fastgen_small "
                               "or decode_is_independent"],
-                       env=env, capture_output=True, text=True, timeout=900)
+                       capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
@@ -718,57 +718,53 @@ def test_layout_compact_matches_the_two_calls(S, d, dt):
 def test_grid_stride_compaction_on_workloads():
     """The grid-stride compaction kernel (forced here; the one-wave kernel is the default)
     gives the same bit-exact packed caches."""
-    import os
     import subprocess
     import sys
-    env = dict(os.environ, KVC_COMPACT_PATH="grid")
-    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+    forced = ['--kvc-path', 'compact=grid']
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider", *forced,
                         "-k", "llama8b_shape_small_context or zigzag_small or fastgen_small or chunk_small"],
-                       env=env, capture_output=True, text=True, timeout=900)
+                       capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
 def test_two_launch_scoring_on_fused_workloads():
     """Workloads whose scoring runs fused in slot clusters by default pass the same checks
     through the two-launch form (pass 1, merge, pass 2), forced here."""
-    import os
     import subprocess
     import sys
-    env = dict(os.environ, KVC_SCORE_PATH="twopass")
-    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+    forced = ['--kvc-path', 'score=twopass']
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider", *forced,
                         "-k", "llama8b_shape_small_context or chunk_small or llama8b_full_size or "
                               "ragged_context_lengths or gqa_group_sizes or head_dims_and_dtypes or window_of_one"],
-                       env=env, capture_output=True, text=True, timeout=900)
+                       capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
 def test_token_split_decode_on_few_slot_workloads():
     """Workloads with few slots decode through thread-block clusters by default; the
     token-range split (forced here) passes the same oracle checks."""
-    import os
     import subprocess
     import sys
-    env = dict(os.environ, KVC_DECODE_SPLIT="tokens")
-    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+    forced = ['--kvc-path', 'decode_split=tokens']
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider", *forced,
                         "-k", "llama8b_shape_small_context or zigzag_small or chunk_small or fastgen_small "
                               "or decode_is_independent or separate_append or fused_append_decode_overflow "
                               "or ragged_context_lengths or gqa_group_sizes"],
-                       env=env, capture_output=True, text=True, timeout=900)
+                       capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
 def test_tcgen05_decode_path_on_bf16_workloads():
     """The tcgen05 decode (opt-in cross-check path, d = 128) passes the same oracle checks,
     including full-size llama8b and the fused-append overflow case."""
-    import os
     import subprocess
     import sys
-    env = dict(os.environ, KVC_DECODE_PATH="tc")
-    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider",
+    forced = ['--kvc-path', 'decode=tc']
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider", *forced,
                         "-k", "llama8b_shape_small_context or zigzag_small or chunk_small or fastgen_small "
                               "or llama8b_full_size or separate_append or fused_append_decode_overflow "
                               "or ragged_context_lengths or gqa_group_sizes"],
-                       env=env, capture_output=True, text=True, timeout=900)
+                       capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
@@ -1002,3 +998,21 @@ def test_fastgen_sliding_local_window_matches_oracle():
             assert int(pipe.len[s]) == wl.local_window
         for t in range(wl.steps):
             P.check_out(outs[t][s * G:(s + 1) * G], ref.out[(t, s)], "bf16", f"step {t} slot {s}")
+
+
+@pytest.mark.parametrize("case", json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                                            "alloc_examples.json")))["cases"],
+                         ids=lambda c: c["name"])
+def test_allocation_worked_examples_on_gpu(case):
+    """kvc_alloc_budgets on the hand-worked ZigZagKV Eq. 4-6 examples (exact, largest remainder,
+    tied remainders to the lower layer, cap at the context, uniform, floor only)."""
+    import sparse_decode_attention_window_b200 as kvc
+    counts = np.array(case["counts"], dtype=np.int32)
+    nL, spl = counts.shape
+    budgets = torch.full((nL,), -1, dtype=torch.int32, device="cuda")
+    slot_b = torch.full((nL * spl,), -1, dtype=torch.int32, device="cuda")
+    kvc.kvc_alloc_budgets(torch.from_numpy(counts.reshape(-1)).cuda(), nL, spl, case["L"], case["avg"],
+                          case["floor"], budgets, slot_b)
+    kvc.kvc_get_status()
+    assert budgets.cpu().tolist() == case["budgets"]
+    assert slot_b.cpu().tolist() == [b for b in case["budgets"] for _ in range(spl)]
