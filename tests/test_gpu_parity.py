@@ -1016,3 +1016,58 @@ def test_allocation_worked_examples_on_gpu(case):
     kvc.kvc_get_status()
     assert budgets.cpu().tolist() == case["budgets"]
     assert slot_b.cpu().tolist() == [b for b in case["budgets"] for _ in range(spl)]
+
+
+@pytest.mark.parametrize("S,counts,steps", [(40, "ragged", 96), (8, "uniform", 96), (6, [0, 1, 2, 3, 5, 7], 64)])
+def test_chained_append_decode_every_step_matches_oracle(S, counts, steps):
+    """Many chained append + decode launches back to back on one stream (each may start while
+    the previous one drains): every step of every slot matches the oracle's attention over the
+    cache grown by one token per step, and the lengths grow by exactly one per step. Ragged
+    slots (the token split, ranges crossing slots), near-uniform slots (per-slot clusters) and
+    a cache so small that most CTAs have no tokens (every CTA still takes its length ticket)."""
+    import sparse_decode_attention_window_b200 as kvc
+    G, d = 4, 128
+    g = torch.Generator().manual_seed(1000 + S)
+    if counts == "ragged":
+        cnt = torch.randint(0, 600, (S,), generator=g, dtype=torch.int32)
+        cnt[::7] = 0
+    elif counts == "uniform":
+        cnt = torch.randint(990, 1010, (S,), generator=g, dtype=torch.int32)
+    else:
+        cnt = torch.tensor(counts, dtype=torch.int32)
+    sh = kvc.make_shape(S, G, d, int(cnt.max()) + steps, 0, S, 1, torch.bfloat16)
+    count = cnt.cuda()
+    off = torch.empty(S + 1, dtype=torch.int64, device="cuda")
+    cap = torch.empty(S, dtype=torch.int32, device="cuda")
+    kvc.kvc_layout(count, steps, off, cap)
+    rows = int(off[-1])
+    kp = torch.randn(rows, d, generator=g).to(torch.bfloat16).cuda()
+    vp = torch.randn(rows, d, generator=g).to(torch.bfloat16).cuda()
+    kp0, vp0 = kp.cpu(), vp.cpu()
+    q = torch.randn(steps, S * G, d, generator=g).to(torch.bfloat16).cuda()
+    kn = torch.randn(steps, S, d, generator=g).to(torch.bfloat16).cuda()
+    vn = torch.randn(steps, S, d, generator=g).to(torch.bfloat16).cuda()
+    ws = torch.zeros(kvc.kvc_workspace_size(kvc.KVC_WS_DECODE, sh), dtype=torch.uint8, device="cuda")
+    ln = count.clone()
+    o = torch.empty((steps, S * G, d), device="cuda")
+    for t in range(steps):
+        if t > 0:
+            kvc.kvc_append_decode_chain(sh, kn[t], vn[t], q[t], kp, vp, off, cap, count, ln, o[t], ws)
+        else:
+            kvc.kvc_append_decode(sh, kn[t], vn[t], q[t], kp, vp, off, cap, ln, o[t], ws)
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    assert torch.equal(ln, count + steps)
+    offs, oc = _np(off), _np(o)
+    qc, knc, vnc = q.cpu(), kn.cpu(), vn.cpu()
+    for s in range(S):
+        c = int(cnt[s])
+        keys = torch.cat([kp0[offs[s]:offs[s] + c], knc[:, s]])
+        vals = torch.cat([vp0[offs[s]:offs[s] + c], vnc[:, s]])
+        # the appended rows are in the cache, in order
+        np.testing.assert_array_equal(_np(kp[offs[s]:offs[s] + c + steps].view(torch.int16)),
+                                      keys.view(torch.int16).numpy())
+        for t in range(steps):
+            n = c + t + 1
+            ref = O.decode_attention(qc[t, s * G:(s + 1) * G], keys[:n], vals[:n], [0, n], [n], G)
+            P.check_out(oc[t, s * G:(s + 1) * G], ref, "bf16", f"slot {s} step {t}")
