@@ -369,7 +369,10 @@ kvc_status kvc_check_wait_limit(int32_t limit_us, cudaStream_t stream);
  *   callers never call it: with every knob at 0 (the state at load) each call takes
  *   the path its shape selects. Nothing else (no environment variable) changes a path.
  *   knob (KVC_DIAG_*) and choice:
- *     KVC_DIAG_SCORE        0 auto, 1 two-launch tensor-core form, 2 CUDA-core kernels
+ *     KVC_DIAG_SCORE        0 auto, 1 two-launch tensor-core form, 2 CUDA-core kernels,
+ *                           3 the earlier slot-cluster form with 128-key tiles (one launch;
+ *                           two-launch where the slots do not fill the GPU in clusters)
+ *     KVC_DIAG_SCORE_K      0 auto, 1..16: CTAs per slot of the default scoring form
  *     KVC_DIAG_SELECT       0 auto, 1 one CTA per slot
  *     KVC_DIAG_COMPACT      0 auto, 1 grid-stride compaction kernel
  *     KVC_DIAG_DECODE       0 auto, 1 CUDA-core decode, 2 tcgen05 decode (bf16, d = 128)
@@ -383,9 +386,11 @@ kvc_status kvc_check_wait_limit(int32_t limit_us, cudaStream_t stream);
 #define KVC_DIAG_COMPACT 2
 #define KVC_DIAG_DECODE 3
 #define KVC_DIAG_DECODE_SPLIT 4
-#define KVC_DIAG_KNOBS 5
+#define KVC_DIAG_SCORE_K 5
+#define KVC_DIAG_KNOBS 6
 #define KVC_DIAG_SCORE_TWO_PASS 1
 #define KVC_DIAG_SCORE_SIMT 2
+#define KVC_DIAG_SCORE_CLUSTER 3
 #define KVC_DIAG_SELECT_CTA 1
 #define KVC_DIAG_COMPACT_GRID 1
 #define KVC_DIAG_DECODE_SIMT 1

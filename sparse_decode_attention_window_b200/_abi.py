@@ -29,11 +29,12 @@ EXPORTS = ["kvc_score", "kvc_select", "kvc_alloc_budgets", "kvc_layout", "kvc_co
 
 # kvc_diag_set_path knobs and choices (cross-checks only)
 KVC_DIAG = {
-    "score": (0, {"auto": 0, "twopass": 1, "simt": 2}),
+    "score": (0, {"auto": 0, "twopass": 1, "simt": 2, "cluster": 3}),
     "select": (1, {"auto": 0, "cta": 1}),
     "compact": (2, {"auto": 0, "grid": 1}),
     "decode": (3, {"auto": 0, "simt": 1, "tc": 2}),
     "decode_split": (4, {"auto": 0, "tokens": 1}),
+    "score_k": (5, {"auto": 0, **{str(k): k for k in range(1, 17)}}),
 }
 
 

@@ -17,6 +17,7 @@
 #include "score_simt.cuh"
 #include "cache.cuh"
 #include "score_sm100.cuh"
+#include "score_cl.cuh"
 #include "select.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
@@ -116,8 +117,13 @@ int diag(int knob) { return g_diag[knob].load(std::memory_order_relaxed); }
 
 // bf16 scoring on the CUDA-core kernels
 bool force_simt() { return diag(KVC_DIAG_SCORE) == KVC_DIAG_SCORE_SIMT; }
-// tensor-core scoring in its two-launch form where the fused slot-cluster kernel would run
+// tensor-core scoring in its two-launch form (pass 1, merge, pass 2)
 bool force_two_pass_score() { return diag(KVC_DIAG_SCORE) == KVC_DIAG_SCORE_TWO_PASS; }
+// tensor-core scoring in its earlier slot-cluster form with 128-key tiles (both passes in one
+// launch, few slots), else two-launch
+bool force_cluster_score() { return diag(KVC_DIAG_SCORE) == KVC_DIAG_SCORE_CLUSTER; }
+// CTAs per slot of the slot-cluster scoring (0: chosen from the shape)
+int diag_cluster_k() { return diag(KVC_DIAG_SCORE_K); }
 // selection at one CTA per slot where slot clusters would run
 bool force_cta_select() { return diag(KVC_DIAG_SELECT) == KVC_DIAG_SELECT_CTA; }
 // the grid-stride compaction kernel instead of the one-wave kernel
@@ -518,8 +524,12 @@ kvc_status kvc_score(const kvc_shape* shape, const void* q_win, const void* k, c
 
   if (kvc::tc_supported(shape, di->cc_major, di->cc_minor) && !force_simt()) {
     unsigned nl = 0;
-    rc = kvc::tc_score(shape, q_win, k, chunk_end, C, row_lse, score, part, lse, wsb + w.keys_off, di->sms, stream,
-                       &fail, &nl, force_two_pass_score());
+    if (force_two_pass_score() || force_cluster_score() || !kvc::cl_takes(shape, Cc, di->sms, diag_cluster_k()))
+      rc = kvc::tc_score(shape, q_win, k, chunk_end, C, row_lse, score, part, lse, wsb + w.keys_off, di->sms, stream,
+                         &fail, &nl, force_two_pass_score());
+    else
+      rc = kvc::tc_score_cl(shape, q_win, k, chunk_end, C, row_lse, score, lse, wsb + w.keys_off, di->sms, stream,
+                            &fail, &nl, diag_cluster_k());
     count_launches(nl);
     if (rc != KVC_OK) return rc;
     return check_launch("kvc_score");
@@ -696,7 +706,7 @@ __global__ void wait_limit_probe_kernel(unsigned long long limit_ns) {
 }  // namespace kvc
 
 kvc_status kvc_diag_set_path(int32_t knob, int32_t choice) {
-  static const int n_choices[KVC_DIAG_KNOBS] = {3, 2, 2, 3, 2};
+  static const int n_choices[KVC_DIAG_KNOBS] = {4, 2, 2, 3, 2, 17};
   if (knob < 0 || knob >= KVC_DIAG_KNOBS) return fail(KVC_ERR_INVALID_ARG, "kvc_diag_set_path: unknown knob %d", knob);
   if (choice < 0 || choice >= n_choices[knob])
     return fail(KVC_ERR_INVALID_ARG, "kvc_diag_set_path: choice %d not in [0, %d) for knob %d", choice,

@@ -727,15 +727,21 @@ def test_grid_stride_compaction_on_workloads():
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
-def test_two_launch_scoring_on_fused_workloads():
-    """Workloads whose scoring runs fused in slot clusters by default pass the same checks
-    through the two-launch form (pass 1, merge, pass 2), forced here."""
+@pytest.mark.parametrize("forced", [["--kvc-path", "score=twopass"], ["--kvc-path", "score=cluster"],
+                                    ["--kvc-path", "score_k=1"], ["--kvc-path", "score_k=3"],
+                                    ["--kvc-path", "score_k=16"]],
+                         ids=["two_launch", "cluster_128key_tiles", "one_cta_per_slot", "three_ctas_per_slot",
+                              "sixteen_ctas_per_slot"])
+def test_other_scoring_forms_on_workloads(forced):
+    """Workloads whose scoring runs in 256-key slot clusters by default pass the same checks
+    through the two-launch form (pass 1, merge, pass 2), the earlier slot-cluster form with
+    128-key tiles, and the slot clusters at 1, 3 and 16 CTAs per slot, each forced here."""
     import subprocess
     import sys
-    forced = ['--kvc-path', 'score=twopass']
     r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-q", "-m", "gpu", "-p", "no:cacheprovider", *forced,
                         "-k", "llama8b_shape_small_context or chunk_small or llama8b_full_size or "
-                              "ragged_context_lengths or gqa_group_sizes or head_dims_and_dtypes or window_of_one"],
+                              "ragged_context_lengths or gqa_group_sizes or head_dims_and_dtypes or window_of_one or "
+                              "prefill_row_normalisers or chunk_full_size"],
                        capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
