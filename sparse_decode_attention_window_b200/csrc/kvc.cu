@@ -647,12 +647,14 @@ kvc_status launch_select(kvc::SelectParams p, int S, int N, cudaStream_t stream,
       return fail(KVC_ERR_CUDA, "%s: launch: %s", what, cudaGetErrorString(e));
     }
   } else {
-    // More slots than SMs: without the key cache two 1024-thread CTAs fit on an SM, so the
-    // slots run in one wave (the scores are re-read from L2 each pass); otherwise cache them.
-    p.key_cap = S > di->sms ? 0 : kvc::select_key_cap(p.L, p.C);
+    // More slots than SMs: no key cache and 512-thread CTAs, so two share an SM (64
+    // registers a thread) and the slots run in one wave, the scores re-read from L2 each
+    // pass; otherwise one 1024-thread CTA per slot caches its keys.
+    const bool many = S > di->sms;
+    p.key_cap = many ? 0 : kvc::select_key_cap(p.L, p.C);
     smem = kvc::select_smem_bytes(p.key_cap);
     if ((rc = set_smem(kvc::select_kernel, smem, what)) != KVC_OK) return rc;
-    kvc::select_kernel<<<S, kvc::SEL_THREADS, smem, stream>>>(p);
+    kvc::select_kernel<<<S, many ? kvc::SEL_THREADS / 2 : kvc::SEL_THREADS, smem, stream>>>(p);
   }
   count_launches(1);
   return check_launch(what);

@@ -44,6 +44,8 @@ KVC_DEV uint32_t order_key(float f) {
   uint32_t b = __float_as_uint(f);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
+// The score whose order_key is k (the mapping is a bijection on bit patterns).
+KVC_DEV float key_score(uint32_t k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k); }
 
 // floor(max(v, 0) * 2^fx) as an integer, exactly: the fp32 significand shifted by the
 // scaled exponent (no floating-point rounding). The scale is chosen from the slot's
@@ -166,13 +168,38 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     }
   }
   auto raw_key = [&](int n) -> uint32_t { return n >= N - n_local ? 0xffffffffu : order_key(sc[n]); };
+  // Keys are read four consecutive ones per thread with one 16-byte load where the slot's
+  // scores are 16-byte aligned (the passes are bound by the latency of these loads when the
+  // keys are not cached in shared memory).
+  const bool vec = ((reinterpret_cast<uintptr_t>(sc) & 15u) == 0);
+  auto keys4 = [&](int n0, uint32_t* k4) {
+    if (cached) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) k4[i] = n0 + i < N ? keys[n0 + i] : 0u;
+    } else if (vec && n0 + 3 < N && n0 + 3 < N - n_local) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(sc + n0));
+      k4[0] = order_key(f.x);
+      k4[1] = order_key(f.y);
+      k4[2] = order_key(f.z);
+      k4[3] = order_key(f.w);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) k4[i] = n0 + i < N ? raw_key(n0 + i) : 0u;
+    }
+  };
   if (cached)
     for (int n = tid; n < N; n += blockDim.x) keys[n] = raw_key(n);
   // weights
   int fx = 0;
   if (massc) {
     float mx = 0.f;
-    for (int n = tid; n < N; n += blockDim.x) mx = fmaxf(mx, sc[n]);
+    for (int n0 = tid * 4; n0 < N; n0 += blockDim.x * 4) {
+      uint32_t k4[4];
+      keys4(n0, k4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (n0 + i < N) mx = fmaxf(mx, key_score(k4[i]));
+    }
     mx = warp_max(mx);
     if ((tid & 31) == 0) sh.scan32[tid >> 5] = __float_as_uint(mx);
     __syncthreads();
@@ -188,11 +215,10 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     fx = sh.fixed_exp;
   }
   auto key_of = [&](int n) -> uint32_t { return cached ? keys[n] : raw_key(n); };
-  auto weight_of = [&](int n) -> unsigned long long {
+  // the weight of key n (MASS_COUNT: its score, recovered from the key)
+  auto weight_of = [&](int n, uint32_t key) -> unsigned long long {
     if (chunk) return (unsigned long long)(ce[n] - (n > 0 ? ce[n - 1] : -1));
-    if (massc) {
-      return fixed_weight(sc[n], fx);
-    }
+    if (massc) return fixed_weight(key_score(key), fx);
     return 1ull;
   };
 
@@ -222,23 +248,21 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     const int nb = pass == 2 ? 1024 : 2048;
     for (int b = tid; b < nb; b += blockDim.x) { sh.hcnt[b] = 0; sh.hwl[b] = 0; sh.hwh[b] = 0; }
     __syncthreads();
-    for (int base = 0; base < N; base += blockDim.x) {
-      const int n = base + tid;
-      bool match = false;
-      uint32_t bin = 0;
-      unsigned long long wt = 0;
-      if (n < N) {
-        uint32_t key = key_of(n);
-        match = (key & pmask) == prefix;
-        bin = (key >> shift) & (nb - 1);
-        if (match) wt = weight_of(n);
-      }
-      // one shared atomic per key and word (grouping a warp's keys by bin with match.any
-      // costs more when they spread over many bins); top-B: every weight is 1, the count
-      // is the weight
-      if (match) {
-        atomicAdd(&sh.hcnt[bin], 1u);
-        if (!unit) bin_add_u64(&sh.hwl[bin], &sh.hwh[bin], wt);
+    for (int n0 = tid * 4; n0 < N; n0 += blockDim.x * 4) {
+      uint32_t k4[4];
+      keys4(n0, k4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int n = n0 + i;
+        const uint32_t key = k4[i];
+        // one shared atomic per key and word (grouping a warp's keys by bin with match.any
+        // costs more when they spread over many bins); top-B: every weight is 1, the count
+        // is the weight
+        if (n < N && (key & pmask) == prefix) {
+          const uint32_t bin = (key >> shift) & (nb - 1);
+          atomicAdd(&sh.hcnt[bin], 1u);
+          if (!unit) bin_add_u64(&sh.hwl[bin], &sh.hwh[bin], weight_of(n, key));
+        }
       }
     }
     __syncthreads();
@@ -310,7 +334,8 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     unsigned long long carry = 0;
     for (int base = 0; base < N; base += blockDim.x) {
       const int n = base + tid;
-      unsigned long long wt = (n < N && key_of(n) == T) ? weight_of(n) : 0ull, tot;
+      const uint32_t key = n < N ? key_of(n) : 0u;
+      unsigned long long wt = (n < N && key == T) ? weight_of(n, key) : 0ull, tot;
       unsigned long long before = carry + block_exclusive_scan<unsigned long long>(wt, sh.scan64, &tot);
       if (wt > 0 && before < need && before + wt >= need) sh.s_sel = before + wt;
       carry += tot;
@@ -331,10 +356,11 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams a) {
     uint32_t kk[SEL_IT], ww[SEL_IT];
     uint32_t g_loc = 0, t_loc = 0;
 #pragma unroll
+    for (int i = 0; i < SEL_IT; i += 4) keys4(n0 + i, kk + i);
+#pragma unroll
     for (int i = 0; i < SEL_IT; ++i) {
       const int n = n0 + i;
-      kk[i] = n < N ? key_of(n) : 0u;
-      ww[i] = (n < N && kk[i] >= T) ? (uint32_t)weight_of(n) : 0u;
+      ww[i] = (n < N && kk[i] >= T) ? (uint32_t)weight_of(n, kk[i]) : 0u;
       if (kk[i] > T) g_loc += ww[i];
       else if (kk[i] == T) t_loc += ww[i];
     }
@@ -407,9 +433,6 @@ struct SelClShared {
   uint32_t sel_bin, cnt_above_bin, bin_c;
   unsigned long long w_above_bin, bin_w;
 };
-
-// The fp32 score whose order_key is k.
-KVC_DEV float key_score(uint32_t k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k); }
 
 KVC_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.aligned;" ::: "memory"); }
 

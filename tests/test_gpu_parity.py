@@ -226,7 +226,7 @@ def test_mass_count_closed_forms_on_gpu():
 
 
 # slot counts whose selection runs in clusters of 16, 8, 4 and 2 CTAs per slot, and at one CTA per slot
-SELECT_SHAPES = [(1, 4096), (3, 2048), (9, 2048), (18, 1000), (37, 3000), (60, 777), (150, 300)]
+SELECT_SHAPES = [(1, 4096), (3, 2048), (9, 2048), (18, 1000), (37, 3000), (60, 777), (150, 300), (200, 777)]
 
 
 @pytest.mark.parametrize("S,N", SELECT_SHAPES)
@@ -270,6 +270,36 @@ def test_selection_policies_over_slot_counts(S, N):
         else:
             want = O.full_indices(N)
         np.testing.assert_array_equal(got, want, err_msg=f"slot {s} policy {k}")
+
+
+@pytest.mark.parametrize("S,N,bound_holds", [(200, 4100, True), (200, 4100, False), (160, 777, True)])
+def test_many_slot_mass_count_and_top_b(S, N, bound_holds):
+    """More slots than SMs (two 512-thread CTAs per SM, keys re-read from L2 four at a time):
+    LMBA counts within the tie band and top-B sets within the tie band of the oracle, for
+    window-like scores (each slot's scores sum to G w, none above it) and for scores scaled far
+    above that, on 16-byte-aligned and unaligned score rows (N = 777)."""
+    import sparse_decode_attention_window_b200 as kvc
+    G, w = 4, 8
+    g = torch.Generator().manual_seed(S * 31 + N)
+    raw = torch.softmax(torch.randn((S, N), generator=g) * 3, dim=1) * (G * w)   # sums to G w per slot
+    sc = (raw if bound_holds else raw * 40).float()
+    if bound_holds:
+        assert float(sc.max()) <= G * w
+    sh = kvc.make_shape(S, G, 64, N, w, 1, S, torch.bfloat16)
+    pol = torch.tensor([kvc.KVC_POL_MASS_COUNT if s % 2 else kvc.KVC_POL_TOPB for s in range(S)], dtype=torch.int8)
+    bud = torch.randint(1, N, (S,), generator=g, dtype=torch.int32)
+    idx = torch.full((S, N), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((S,), -1, dtype=torch.int32, device="cuda")
+    kvc.kvc_select(sh, sc.cuda(), pol.cuda(), bud.cuda(), idx, cnt, mass=0.9)
+    torch.cuda.synchronize()
+    kvc.kvc_get_status()
+    idx, cnt = _np(idx), _np(cnt)
+    sc64 = sc.double().numpy()
+    for s in range(S):
+        if s % 2:
+            P.check_mass_count(int(cnt[s]), sc64[s], 0.9, f"slot {s}")
+        else:
+            P.check_topb(idx[s, :cnt[s]].astype(np.int64), sc64[s], int(bud[s]), f"slot {s}")
 
 
 @pytest.mark.parametrize("S,C", [(1, 3000), (5, 1200), (9, 2048), (40, 700), (150, 200)])
